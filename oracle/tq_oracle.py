@@ -1,0 +1,361 @@
+"""Plain, slow, fp64 CPU oracle for TurboQuant-style KV-cache compression.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
+only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it.  It shares no code, tables or
+constants with the CUDA library; every function is written from the pages'
+definitions in the most direct form (dense matrices, explicit loops where the
+definition is a loop, numpy/BLAS only as a step primitive).
+
+Pages cited (by title and section):
+  [llama-tq]      "llama-tq: 让大模型在消费级显卡上跑起10万token长上下文的技术突破",
+                  section "KV缓存量化的技术困境与TurboQuant的解决方案" (K cache:
+                  randomized Hadamard + Lloyd-Max; Q.K in the Hadamard domain,
+                  no K dequantisation; V "v1 codebook" sub-family).
+  [tq+ README]    "TheTom/llama-cpp-turboquant" README, table "量化类型"
+                  (all turbo formats: WHT rotation then polar codebook
+                  quantisation on 128-element blocks) and "压缩策略" (sparse-V
+                  dequant: skip V where the softmax weight is below a threshold).
+  [TurboQuant+]   "TurboQuant+: 面向生产环境的LLM KV缓存与权重量化技术", sections
+                  "Walsh-Hadamard变换" and "注意力门控稀疏V解压" (skipped V is
+                  treated as zero).
+  [TQ article]    intelliparadigm TurboQuant article, §3.2 "随机哈达玛变换详解"
+                  (H_random = D x H, D diagonal random +-1, fast WHT O(d log d)),
+                  §3.3 "Lloyd-Max量化算法" (init centres, assign to nearest,
+                  centre = mean of its points, repeat), §4.1 table (bits/ratio).
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  * rotation order H.D (signs first, then the unnormalised Sylvester WHT);
+  * sign vector from SplitMix64 (Steele, Lea, Flood 2014), state = seed,
+    s_i = -1 when the top bit of the i-th output is set;
+  * one sign vector for K, V, every block, head and batch entry;
+  * per-block norm = the raw fp64 L2 norm of the input block, stored as fp16
+    (round to nearest even); direction u = y / n with the unrounded norm;
+  * Lloyd-Max run on the N(0,1) density (not on samples); boundaries are
+    midpoints; the fp32-rounded boundaries decide the codes; a value equal to a
+    boundary goes to the lower index; a zero block gives index L/2 - 1;
+  * codes packed LSB-first into a little-endian bitstream of 16*b bytes;
+  * sparse-V weight = normalised softmax weight exp(s - LSE); positions below
+    the threshold contribute zero and the rest are not renormalised.
+"""
+from __future__ import annotations
+
+import math
+from statistics import NormalDist
+
+import numpy as np
+
+BLOCK = 128
+_MASK64 = (1 << 64) - 1
+
+# ---------------------------------------------------------------------------
+# Rotation: H_random = H . diag(s)   ([TQ article] §3.2; [TurboQuant+] WHT)
+# ---------------------------------------------------------------------------
+
+
+def splitmix64(seed: int, count: int) -> list[int]:
+    """The first ``count`` outputs of SplitMix64 started from state ``seed``.
+
+    Published generator (Steele, Lea, Flood, OOPSLA 2014): the state advances
+    by the golden-ratio increment and each output is the state passed through
+    two xor-shift-multiply rounds and a final xor-shift.
+    """
+    state = seed & _MASK64
+    out = []
+    for _ in range(count):
+        state = (state + 0x9E3779B97F4A7C15) & _MASK64
+        z = state
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK64
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK64
+        z = z ^ (z >> 31)
+        out.append(z)
+    return out
+
+
+def sign_vector(seed: int, d: int = BLOCK) -> np.ndarray:
+    """The random +-1 diagonal of D ([TQ article] §3.2), as fp64."""
+    return np.array([-1.0 if (z >> 63) else 1.0 for z in splitmix64(seed, d)])
+
+
+def hadamard(d: int = BLOCK) -> np.ndarray:
+    """Unnormalised Sylvester Hadamard matrix, H[i, j] = (-1)^popcount(i & j)."""
+    h = np.empty((d, d))
+    for i in range(d):
+        for j in range(d):
+            h[i, j] = -1.0 if bin(i & j).count("1") % 2 else 1.0
+    return h
+
+
+def rotate(x: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """y = H . diag(s) . x for every 128-element block along the last axis.
+
+    Dense matrix product, not a butterfly (the oracle must not share the fast
+    transform's structure with the kernels).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    assert d % BLOCK == 0
+    blocks = x.reshape(*x.shape[:-1], d // BLOCK, BLOCK)
+    y = (blocks * signs) @ hadamard(BLOCK).T
+    return y.reshape(x.shape)
+
+
+def unrotate(y: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`rotate`: x = diag(s) . H . y / d (since H.H^T = d.I)."""
+    y = np.asarray(y, dtype=np.float64)
+    d = y.shape[-1]
+    blocks = y.reshape(*y.shape[:-1], d // BLOCK, BLOCK)
+    x = (blocks @ hadamard(BLOCK).T) * signs / BLOCK
+    return x.reshape(y.shape)
+
+
+# ---------------------------------------------------------------------------
+# Lloyd-Max codebook for N(0,1)   ([TQ article] §3.3; [llama-tq] K cache)
+# ---------------------------------------------------------------------------
+
+
+def _phi(t: float) -> float:
+    if math.isinf(t):
+        return 0.0
+    return math.exp(-0.5 * t * t) / math.sqrt(2.0 * math.pi)
+
+
+def _Phi(t: float) -> float:
+    if t == -math.inf:
+        return 0.0
+    if t == math.inf:
+        return 1.0
+    return 0.5 * math.erfc(-t / math.sqrt(2.0))
+
+
+def lloyd_max_gaussian(bits: int, tol: float = 1e-13, max_iter: int = 200000):
+    """Lloyd-Max quantiser of the N(0,1) density, in fp64.
+
+    Follows the four steps of [TQ article] §3.3 with the continuous density in
+    place of data points:
+      1. initial centres c_j = Phi^-1((j + 1/2) / L);
+      2. assignment to the nearest centre = cells bounded by the midpoints
+         t_j = (c_j + c_{j+1}) / 2 (t_{-1} = -inf, t_{L-1} = +inf);
+      3. each centre becomes the mean of its cell,
+         c_j = (phi(t_{j-1}) - phi(t_j)) / (Phi(t_j) - Phi(t_{j-1}));
+      4. repeat 2-3 until no centre moves by ``tol`` or more.
+    Returns (centroids[L], boundaries[L-1]) in fp64.
+    """
+    levels = 1 << bits
+    nd = NormalDist()
+    c = [nd.inv_cdf((j + 0.5) / levels) for j in range(levels)]
+    for _ in range(max_iter):
+        t = [(c[j] + c[j + 1]) / 2.0 for j in range(levels - 1)]
+        edges = [-math.inf] + t + [math.inf]
+        new = [(_phi(edges[j]) - _phi(edges[j + 1])) / (_Phi(edges[j + 1]) - _Phi(edges[j]))
+               for j in range(levels)]
+        delta = max(abs(a - b) for a, b in zip(new, c))
+        c = new
+        if delta < tol:
+            break
+    t = [(c[j] + c[j + 1]) / 2.0 for j in range(levels - 1)]
+    return np.array(c), np.array(t)
+
+
+def codebook_f32(bits: int):
+    """The codebook as the kernels use it: fp32 centroids and boundaries."""
+    c, t = lloyd_max_gaussian(bits)
+    return c.astype(np.float32), t.astype(np.float32)
+
+
+def gaussian_distortion(centroids, boundaries) -> float:
+    """E[(X - Q(X))^2] for X ~ N(0,1), from the closed-form cell moments."""
+    c = [float(v) for v in centroids]
+    edges = [-math.inf] + [float(v) for v in boundaries] + [math.inf]
+    total = 0.0
+    for j, cj in enumerate(c):
+        a, b = edges[j], edges[j + 1]
+        p = _Phi(b) - _Phi(a)
+        m1 = _phi(a) - _phi(b)                       # integral of x phi(x)
+        m2 = p + (a * _phi(a) if not math.isinf(a) else 0.0) \
+            - (b * _phi(b) if not math.isinf(b) else 0.0)  # integral of x^2 phi
+        total += m2 - 2.0 * cj * m1 + cj * cj * p
+    return total
+
+
+# ---------------------------------------------------------------------------
+# Encoder: sign, rotate, norm, quantise, pack ([tq+ README] 量化类型; [llama-tq])
+# ---------------------------------------------------------------------------
+
+
+def quantize(u: np.ndarray, boundaries_f32: np.ndarray) -> np.ndarray:
+    """idx = #{ j : t_j < u }, with t_j the fp32 boundaries read as fp64.
+
+    A value equal to a boundary is not counted, so it takes the lower index.
+    """
+    t = np.asarray(boundaries_f32, dtype=np.float32).astype(np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    idx = np.zeros(u.shape, dtype=np.int64)
+    for tj in t:
+        idx += (tj < u)
+    return idx
+
+
+def pack_codes(idx: np.ndarray, bits: int) -> np.ndarray:
+    """Bit-pack b-bit indices, LSB-first, into a little-endian bitstream.
+
+    ``idx`` has a last axis of 128; the result has a last axis of 16*bits
+    bytes.  Index i occupies stream bits [b*i, b*i + b).
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    assert idx.shape[-1] == BLOCK
+    flat = idx.reshape(-1, BLOCK)
+    out = np.zeros((flat.shape[0], 16 * bits), dtype=np.uint8)
+    for i in range(BLOCK):
+        for k in range(bits):
+            bit = (flat[:, i] >> k) & 1
+            pos = bits * i + k
+            out[:, pos // 8] |= (bit << (pos % 8)).astype(np.uint8)
+    return out.reshape(*idx.shape[:-1], 16 * bits)
+
+
+def unpack_codes(packed: np.ndarray, bits: int) -> np.ndarray:
+    """Inverse of :func:`pack_codes`."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    assert packed.shape[-1] == 16 * bits
+    flat = packed.reshape(-1, 16 * bits).astype(np.int64)
+    idx = np.zeros((flat.shape[0], BLOCK), dtype=np.int64)
+    for i in range(BLOCK):
+        for k in range(bits):
+            pos = bits * i + k
+            idx[:, i] |= ((flat[:, pos // 8] >> (pos % 8)) & 1) << k
+    return idx.reshape(*packed.shape[:-1], BLOCK)
+
+
+def encode(x: np.ndarray, signs: np.ndarray, bits: int, boundaries_f32: np.ndarray):
+    """Encode vectors ``x[..., D]`` (D a multiple of 128).
+
+    Per 128-element block: n = ||x||_2 in fp64; y = H.(s o x); u = y / n
+    (u = 0 for a zero block); idx = quantize(u); codes = pack(idx).
+    Returns (codes[..., D/128, 16*bits] uint8, norms[..., D/128] fp16,
+    u[..., D/128, 128] fp64) -- u is returned so tests can measure distances
+    to decision boundaries.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    nb = d // BLOCK
+    blocks = x.reshape(*x.shape[:-1], nb, BLOCK)
+    n = np.sqrt(np.sum(blocks * blocks, axis=-1))
+    y = rotate(blocks, signs)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        u = np.where(n[..., None] > 0, y / n[..., None], 0.0)
+    idx = quantize(u, boundaries_f32)
+    return pack_codes(idx, bits), n.astype(np.float16), u
+
+
+def dequantize(codes: np.ndarray, norms_f16: np.ndarray, bits: int,
+               centroids_f32: np.ndarray, signs: np.ndarray) -> np.ndarray:
+    """x~ = (n^ / d) . diag(s) . H . c[idx] per block, n^ the stored fp16 norm."""
+    idx = unpack_codes(codes, bits)                      # [..., nb, 128]
+    c = np.asarray(centroids_f32, dtype=np.float32).astype(np.float64)[idx]
+    nhat = np.asarray(norms_f16, dtype=np.float16).astype(np.float64)
+    xt = unrotate(c, signs) * nhat[..., None]            # unrotate divides by d
+    return xt.reshape(*xt.shape[:-2], xt.shape[-2] * BLOCK)
+
+
+# ---------------------------------------------------------------------------
+# Decode attention
+# ---------------------------------------------------------------------------
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_lens, scale: float,
+              sparse_thr: float = 0.0) -> np.ndarray:
+    """Single-token softmax attention in fp64 on dense K/V.
+
+    q: [B, Hq, D]; k, v: [B, Hkv, S, D]; q-head h reads kv-head h // (Hq/Hkv).
+    w = softmax(scale . q.k_t) over t < seq_lens[b] (max-subtracted, fp64).
+    Sparse-V ([tq+ README] 压缩策略; [TurboQuant+] 注意力门控稀疏V解压): with
+    sparse_thr > 0, positions whose normalised weight w_t is below the
+    threshold contribute zero and the kept weights are not renormalised.
+    A sequence of length 0 gives a zero output.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    bsz, hq, d = q.shape
+    hkv = k.shape[1]
+    group = hq // hkv
+    out = np.zeros((bsz, hq, d))
+    for b in range(bsz):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        for h in range(hq):
+            kv = h // group
+            s = scale * (k[b, kv, :n] @ q[b, h])
+            w = np.exp(s - s.max())
+            w = w / w.sum()
+            if sparse_thr > 0:
+                w = np.where(w < sparse_thr, 0.0, w)
+            out[b, h] = w @ v[b, kv, :n]
+    return out
+
+
+def decode_dequant(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale,
+                   k_bits, v_bits, k_centroids, v_centroids, signs, sparse_thr=0.0):
+    """Formulation A: dequantise the whole cache, then plain attention."""
+    kt = dequantize(k_codes, k_norms, k_bits, k_centroids, signs)
+    vt = dequantize(v_codes, v_norms, v_bits, v_centroids, signs)
+    return attention(q, kt, vt, seq_lens, scale, sparse_thr)
+
+
+def decode_rotated(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale,
+                   k_bits, v_bits, k_centroids, v_centroids, signs, sparse_thr=0.0):
+    """Formulation B: the Hadamard-domain steps, in fp64.
+
+    q^ = H.(s o q) per block (Q rotated once, [llama-tq] K cache);
+    s_t = scale . sum_blk (nK_t,blk / d) . q^_blk . cK[idx_t,blk] (no K
+    dequantisation); w = softmax(s); V summed in the rotated domain,
+    acc = sum_t w_t (nV_t,blk / d) cV[idx_t,blk]; one inverse rotation per
+    head, o = s o (H.acc) per block.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    bsz, hq, d = q.shape
+    hkv = k_codes.shape[1]
+    group = hq // hkv
+    nb = d // BLOCK
+    qhat = rotate(q, signs).reshape(bsz, hq, nb, BLOCK)
+    ck = np.asarray(k_centroids, dtype=np.float32).astype(np.float64)[unpack_codes(k_codes, k_bits)]
+    cv = np.asarray(v_centroids, dtype=np.float32).astype(np.float64)[unpack_codes(v_codes, v_bits)]
+    nk = np.asarray(k_norms, dtype=np.float16).astype(np.float64) / BLOCK
+    nv = np.asarray(v_norms, dtype=np.float16).astype(np.float64) / BLOCK
+    h_mat = hadamard(BLOCK)
+    out = np.zeros((bsz, hq, d))
+    for b in range(bsz):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        for h in range(hq):
+            kv = h // group
+            # [n, nb] block dot products, weighted by the block norms.
+            dots = np.einsum("tbi,bi->tb", ck[b, kv, :n], qhat[b, h])
+            s = scale * np.sum(nk[b, kv, :n] * dots, axis=1)
+            w = np.exp(s - s.max())
+            w = w / w.sum()
+            if sparse_thr > 0:
+                w = np.where(w < sparse_thr, 0.0, w)
+            acc = np.einsum("t,tb,tbi->bi", w, nv[b, kv, :n], cv[b, kv, :n])
+            o = (acc @ h_mat.T) * signs
+            out[b, h] = o.reshape(d)
+    return out
+
+
+def sparse_skip_fraction(q, k, seq_lens, scale, thr, group):
+    """Fraction of (q-head, position) pairs whose normalised weight is < thr."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    skipped = total = 0
+    for b in range(q.shape[0]):
+        n = int(seq_lens[b])
+        for h in range(q.shape[1]):
+            s = scale * (k[b, h // group, :n] @ q[b, h])
+            w = np.exp(s - s.max())
+            w /= w.sum()
+            skipped += int(np.sum(w < thr))
+            total += n
+    return skipped / max(total, 1)

@@ -1,0 +1,303 @@
+"""Pins of the CPU oracle to facts fixed outside it (CPU only).
+
+Each test checks one oracle function against something other than itself: a
+closed form, an invariant of the mathematics, a published table, a library
+routine, or brute force.  A plausible slip in the oracle (a dropped term, a
+wrong sign or index, a transposed operand) fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy import integrate, stats
+
+from oracle import tq_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_max():
+    table = {}
+    with open(os.path.join(GOLDEN, "max1960_gaussian.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            lv, kind, vals = [p.strip() for p in line.split("|")]
+            table[(int(lv), kind)] = [float(v) for v in vals.split()]
+    return table
+
+
+def _fwht(x):
+    """Independent in-place butterfly Walsh-Hadamard transform (unnormalised)."""
+    x = np.array(x, dtype=np.float64)
+    h = 1
+    while h < x.shape[-1]:
+        for i in range(0, x.shape[-1], 2 * h):
+            a = x[..., i:i + h].copy()
+            b = x[..., i + h:i + 2 * h].copy()
+            x[..., i:i + h] = a + b
+            x[..., i + h:i + 2 * h] = a - b
+        h *= 2
+    return x
+
+
+# --------------------------------------------------------------- rotation ---
+
+def test_hadamard_orthogonal_exact():
+    h = O.hadamard(128)
+    assert np.array_equal(h @ h.T, 128.0 * np.eye(128))
+    assert np.array_equal(h, h.T)
+    assert set(np.unique(h)) == {-1.0, 1.0}
+
+
+def test_dense_rotation_equals_butterfly():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((7, 256))
+    s = O.sign_vector(5)
+    dense = O.rotate(x, s)
+    fast = np.concatenate([_fwht(s * x[:, :128]), _fwht(s * x[:, 128:])], axis=1)
+    assert np.max(np.abs(dense - fast)) <= 1e-12 * np.max(np.abs(fast))
+
+
+def test_rotation_preserves_geometry_up_to_d():
+    rng = np.random.default_rng(2)
+    x, y = rng.standard_normal((2, 128))
+    s = O.sign_vector(0)
+    rx, ry = O.rotate(x, s), O.rotate(y, s)
+    assert math.isclose(rx @ ry, 128.0 * (x @ y), rel_tol=1e-12, abs_tol=1e-9)
+    assert math.isclose(np.linalg.norm(rx), math.sqrt(128) * np.linalg.norm(x), rel_tol=1e-12)
+    assert np.allclose(O.unrotate(rx, s), x, atol=1e-12)
+
+
+def test_splitmix64_published_check_values():
+    with open(os.path.join(GOLDEN, "splitmix64_seed1234567.txt")) as f:
+        want = [int(l) for l in f if l.strip() and not l.startswith("#")]
+    assert O.splitmix64(1234567, 5) == want
+
+
+def test_sign_vector_is_top_bit_of_splitmix64():
+    s = O.sign_vector(1234567, 5)
+    with open(os.path.join(GOLDEN, "splitmix64_seed1234567.txt")) as f:
+        want = [int(l) for l in f if l.strip() and not l.startswith("#")]
+    assert list(s) == [-1.0 if w >= 2**63 else 1.0 for w in want]
+    s0 = O.sign_vector(0)
+    assert s0.shape == (128,) and set(np.unique(s0)) == {-1.0, 1.0}
+    assert 40 < np.sum(s0 > 0) < 88
+
+
+# --------------------------------------------------------------- codebook ---
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_codebook_matches_max_1960(bits):
+    table = _golden_max()
+    levels = 1 << bits
+    c, t = O.lloyd_max_gaussian(bits)
+    half = c[levels // 2:]
+    np.testing.assert_allclose(half, table[(levels, "centroids")], rtol=6e-4, atol=6e-4)
+    if (levels, "boundaries") in table:
+        np.testing.assert_allclose(t[levels // 2:], table[(levels, "boundaries")], rtol=6e-4, atol=6e-4)
+    dist = O.gaussian_distortion(c, t)
+    assert math.isclose(dist, table[(levels, "distortion")][0], rel_tol=2e-3)
+
+
+def test_codebook_one_bit_closed_form():
+    c, t = O.lloyd_max_gaussian(1)
+    assert math.isclose(c[1], math.sqrt(2 / math.pi), rel_tol=1e-12)
+    assert c[0] == -c[1] and t[0] == 0.0
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_codebook_fixed_point_conditions_by_quadrature(bits):
+    """Centroid condition checked with numerical quadrature (independent of the
+    closed-form cell moments the oracle iterates); midpoint condition exactly."""
+    c, t = O.lloyd_max_gaussian(bits)
+    levels = len(c)
+    np.testing.assert_allclose(c, -c[::-1], atol=1e-15)
+    np.testing.assert_allclose(t, (c[:-1] + c[1:]) / 2, atol=0)
+    edges = [-np.inf] + list(t) + [np.inf]
+    for j in range(levels):
+        mass = integrate.quad(stats.norm.pdf, edges[j], edges[j + 1], epsabs=1e-14)[0]
+        mom = integrate.quad(lambda x: x * stats.norm.pdf(x), edges[j], edges[j + 1], epsabs=1e-14)[0]
+        assert abs(mom / mass - c[j]) < 1e-9
+
+
+def test_codebook_unique_fixed_point_from_other_init():
+    """N(0,1) is log-concave, so Lloyd-Max has one fixed point: a plain
+    sample-free iteration started from a uniform grid reaches the same one."""
+    for bits in (2, 3, 4):
+        c_ref, _ = O.lloyd_max_gaussian(bits)
+        levels = 1 << bits
+        c = np.linspace(-2.5, 2.5, levels)
+        for _ in range(20000):
+            t = (c[:-1] + c[1:]) / 2
+            e = np.concatenate([[-np.inf], t, [np.inf]])
+            c = (stats.norm.pdf(e[:-1]) - stats.norm.pdf(e[1:])) / (stats.norm.cdf(e[1:]) - stats.norm.cdf(e[:-1]))
+        np.testing.assert_allclose(c, c_ref, atol=1e-9)
+
+
+# -------------------------------------------------------------- quantizer ---
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantizer_is_nearest_centroid(bits):
+    c32, t32 = O.codebook_f32(bits)
+    rng = np.random.default_rng(bits)
+    u = np.concatenate([rng.standard_normal(200000) * 1.5,
+                        np.nextafter(t32.astype(np.float64), np.inf),
+                        np.nextafter(t32.astype(np.float64), -np.inf)])
+    idx = O.quantize(u, t32)
+    brute = np.argmin(np.abs(u[:, None] - c32.astype(np.float64)[None, :]), axis=1)
+    # Away from a boundary the nearest centroid is unique and must agree.
+    far = np.min(np.abs(u[:, None] - t32.astype(np.float64)[None, :]), axis=1) > 1e-6
+    assert np.array_equal(idx[far], brute[far])
+    # Exactly on a boundary: lower index.  Zero maps to L/2 - 1.
+    assert np.array_equal(O.quantize(t32.astype(np.float64), t32), np.arange(len(t32)))
+    assert O.quantize(np.array([0.0]), t32)[0] == (1 << bits) // 2 - 1
+
+
+# ---------------------------------------------------------------- packing ---
+
+def test_pack_known_patterns():
+    idx4 = np.arange(128) % 16
+    p4 = O.pack_codes(idx4, 4)
+    assert p4.shape == (64,)
+    assert list(p4[:3]) == [0x10, 0x32, 0x54]
+    idx2 = np.arange(128) % 4
+    assert np.all(O.pack_codes(idx2, 2) == 0xE4)
+    idx3 = np.arange(128) % 8          # 0..7 repeats: octal 01234567 -> 88 C6 FA
+    p3 = O.pack_codes(idx3, 3)
+    assert p3.shape == (48,)
+    assert list(p3[:6]) == [0x88, 0xC6, 0xFA, 0x88, 0xC6, 0xFA]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_roundtrip_and_bits_per_value(bits):
+    rng = np.random.default_rng(bits)
+    idx = rng.integers(0, 1 << bits, size=(3, 5, 128))
+    packed = O.pack_codes(idx, bits)
+    assert np.array_equal(O.unpack_codes(packed, bits), idx)
+    # Stored bytes per 128-block: 16*b code bytes + one fp16 norm.
+    per_block = packed.shape[-1] + 2
+    assert per_block * 8 / 128 == bits + 16 / 128
+    assert round(16 / (bits + 0.125), 2) == {2: 7.53, 3: 5.12, 4: 3.88}[bits]
+
+
+# ---------------------------------------------------------------- encoder ---
+
+def _sphere_coordinate_mse(centroids, boundaries, d=128):
+    """E[(u - Q(u))^2] where u/sqrt(d) is one coordinate of a uniform point
+    on the unit sphere in R^d: density prop. to (1 - u^2/d)^((d-3)/2)."""
+    r = math.sqrt(d)
+    dens = lambda u: (1 - u * u / d) ** ((d - 3) / 2)
+    z = integrate.quad(dens, -r, r)[0]
+    edges = [-r] + [float(b) for b in boundaries] + [r]
+    tot = 0.0
+    for j, cj in enumerate(centroids):
+        tot += integrate.quad(lambda u: (u - float(cj)) ** 2 * dens(u), edges[j], edges[j + 1])[0]
+    return tot / z
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_reconstruction_mse_matches_sphere_integral(bits):
+    c32, t32 = O.codebook_f32(bits)
+    s = O.sign_vector(0)
+    rng = np.random.default_rng(10 + bits)
+    x = rng.standard_normal((3000, 128)) * rng.lognormal(0, 1, (3000, 1))
+    codes, norms, _ = O.encode(x, s, bits, t32)
+    xt = O.dequantize(codes, norms, bits, c32, s)
+    rel = np.mean(np.sum((x - xt) ** 2, axis=1) / np.sum(x * x, axis=1))
+    want = _sphere_coordinate_mse(c32, t32)
+    assert abs(rel - want) < 0.02 * want, (rel, want)
+
+
+def test_encode_norm_and_zero_block():
+    s = O.sign_vector(3)
+    c32, t32 = O.codebook_f32(3)
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((4, 256))
+    x[2, :128] = 0.0
+    codes, norms, u = O.encode(x, s, 3, t32)
+    assert norms.dtype == np.float16 and norms.shape == (4, 2)
+    np.testing.assert_array_equal(norms, np.linalg.norm(x.reshape(4, 2, 128), axis=-1).astype(np.float16))
+    assert np.all(O.unpack_codes(codes[2, 0], 3) == 3)
+    # u has unit second moment per coordinate: |u|^2 = d exactly.
+    np.testing.assert_allclose(np.sum(u[0] ** 2, axis=-1), 128.0, rtol=1e-12)
+
+
+# -------------------------------------------------------------- attention ---
+
+def _random_cache(rng, bsz, hkv, seq, d, kb, vb, seed=0):
+    s = O.sign_vector(seed)
+    ck, tk = O.codebook_f32(kb)
+    cv, tv = O.codebook_f32(vb)
+    k = rng.standard_normal((bsz, hkv, seq, d))
+    v = rng.standard_normal((bsz, hkv, seq, d))
+    kc, kn, _ = O.encode(k, s, kb, tk)
+    vc, vn, _ = O.encode(v, s, vb, tv)
+    return s, (ck, cv), (k, v), (kc, kn, vc, vn)
+
+
+def test_two_formulations_agree():
+    rng = np.random.default_rng(7)
+    s, (ck, cv), _, (kc, kn, vc, vn) = _random_cache(rng, 2, 2, 40, 256, 3, 2)
+    q = rng.standard_normal((2, 8, 256))
+    lens = [40, 17]
+    for thr in (0.0, 2e-2):
+        a = O.decode_dequant(q, kc, kn, vc, vn, lens, 1 / 16, 3, 2, ck, cv, s, thr)
+        b = O.decode_rotated(q, kc, kn, vc, vn, lens, 1 / 16, 3, 2, ck, cv, s, thr)
+        assert np.max(np.abs(a - b)) <= 1e-10 * np.max(np.abs(a))
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(8)
+    s, (ck, cv), _, (kc, kn, vc, vn) = _random_cache(rng, 1, 1, 6, 128, 4, 4)
+    vt = O.dequantize(vc, vn, 4, cv, s)
+    kt = O.dequantize(kc, kn, 4, ck, s)
+    q = rng.standard_normal((1, 1, 128))
+    dec = lambda qq, lens, thr=0.0: O.decode_rotated(qq, kc, kn, vc, vn, lens, 1 / math.sqrt(128), 4, 4, ck, cv, s, thr)
+    np.testing.assert_allclose(dec(q, [1])[0, 0], vt[0, 0, 0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dec(np.zeros_like(q), [6])[0, 0], vt[0, 0].mean(axis=0), atol=1e-12)
+    assert np.all(dec(q, [0]) == 0)
+    # Two positions, expanded by hand: o = sigmoid(s0 - s1) v0 + sigmoid(s1 - s0) v1.
+    sc = (kt[0, 0, :2] @ q[0, 0]) / math.sqrt(128)
+    w0 = 1 / (1 + math.exp(sc[1] - sc[0]))
+    np.testing.assert_allclose(dec(q, [2])[0, 0], w0 * vt[0, 0, 0] + (1 - w0) * vt[0, 0, 1], atol=1e-12)
+    # One dominant score picks its value vector.
+    qd = 60.0 * kt[0, 0, 3][None, None, :] / np.linalg.norm(kt[0, 0, 3])
+    np.testing.assert_allclose(dec(qd, [6])[0, 0], vt[0, 0, 3], atol=1e-6)
+    # A threshold above every weight leaves nothing; a threshold <= 0 is dense.
+    assert np.all(dec(q, [6], thr=1.01) == 0)
+    np.testing.assert_array_equal(dec(q, [6], thr=-1.0), dec(q, [6]))
+
+
+def test_dense_attention_matches_torch_sdpa():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((2, 8, 128))
+    k = rng.standard_normal((2, 2, 30, 128))
+    v = rng.standard_normal((2, 2, 30, 128))
+    lens = [30, 11]
+    ours = O.attention(q, k, v, lens, 1 / math.sqrt(128))
+    for b in range(2):
+        n = lens[b]
+        qt = torch.tensor(q[b][:, None, :])                         # [Hq, 1, D]
+        kt = torch.tensor(np.repeat(k[b, :, :n], 4, axis=0))       # [Hq, n, D]
+        vt = torch.tensor(np.repeat(v[b, :, :n], 4, axis=0))
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=1 / math.sqrt(128))
+        np.testing.assert_allclose(ours[b], ref[:, 0].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_skip_fraction_matches_gaussian_prediction():
+    """w_t < thr with w_t = exp(s_t - LSE).  Given q, the scores are
+    N(0, sigma^2) with sigma = scale |q|, so LSE ~ log N + sigma^2 / 2 and the
+    skipped fraction is Phi((log(thr N) + sigma^2/2) / sigma)."""
+    rng = np.random.default_rng(11)
+    n, d, heads = 4096, 128, 32
+    thr = 1e-6 * 131072 / n
+    q = rng.standard_normal((1, heads, d))
+    k = rng.standard_normal((1, 1, n, d))
+    got = O.sparse_skip_fraction(q, k, [n], 1 / math.sqrt(d), thr, heads)
+    sig = np.linalg.norm(q[0], axis=1) / math.sqrt(d)
+    pred = np.mean(stats.norm.cdf((np.log(thr * n) + sig ** 2 / 2) / sig))
+    assert abs(got - pred) < 0.004, (got, pred)
+    assert 0.04 < got < 0.09
