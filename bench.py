@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant-style decode step on B200.
+
+One step = the hot path for one generated token of every sequence in the
+batch: encode the newest K/V row of each (batch, kv-head) into the packed cache
+(rotate, norm, quantise, pack) and run single-token decode attention over the
+whole cache (Q rotation, Hadamard-domain scores from codes, online softmax,
+rotated-domain V sum, split merge, inverse rotation).  The newest row is
+written at position seq_len - 1, so every step does identical work.
+
+Default workload: GQA decode, B8, Hq32/Hkv8, D128, S32768, K3/V3, fp16 Q.
+The packed cache (210 MB) rotates over enough copies to exceed 3x L2, so no
+timed step reads warm L2.  Also reported: the encoder alone on the encode-only
+workload (B8, Hkv8, D128, S32768 fp16 in, K3/V2).
+
+Multi-GPU: one process per GPU (torchrun); each rank serves its own batch
+(weak scaling, no collective on the data path); time = max over ranks.
+``--impl reference`` times the CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention KV tokens/s and achieved HBM GB/s (% of ~8 TB/s); encode GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_NAMES = {
+    "gqa": "GQA decode B8 Hq32/Hkv8 D128 S32768 K3/V3 fp16 Q",
+    "long": "long-context decode B1 Hq32/Hkv8 D128 S131072 K4/V2 fp16 Q, sparse-V off",
+    "long_sparse": "long-context decode B1 Hq32/Hkv8 D128 S131072 K4/V2 fp16 Q, sparse-V 1e-6",
+    "ragged": "ragged wide-head decode B4 len U[16384,65536] Hq16/Hkv4 D256 K3/V2, sparse-V 1e-5",
+    "toy": "toy decode B1 Hq1/Hkv1 D128 S256 K4/V4 fp32",
+}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_NAMES), default="gqa")
+    ap.add_argument("--no-encode", action="store_true", help="skip the encode-only measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload(name, rank=0):
+    from quantized_decode_attention_tq_b200 import inputs
+    base = "long" if name == "long_sparse" else name
+    w = inputs.make(base, seed=rank)
+    if name == "long":
+        w.sparse_thr = 0.0
+    return w
+
+
+def kv_bytes(w):
+    nb = w.head_dim // 128
+    per_tok = w.kv_heads * nb * (16 * w.k_bits + 2 + 16 * w.v_bits + 2)
+    return int(np.sum(w.seq_lens)) * per_tok
+
+
+def step_io_bytes(w):
+    q = w.batch * w.q_heads * w.head_dim * np.dtype(w.dtype).itemsize
+    kv_new = 2 * w.batch * w.kv_heads * w.head_dim * np.dtype(w.dtype).itemsize
+    lens = 2 * 4 * w.batch  # seq_lens and start positions
+    out = w.batch * w.q_heads * w.head_dim * 4
+    return q + kv_new + lens, out
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def cpu_oracle_sample(w, kc, kn, vc, vn, units, budget_s=20.0):
+    """Time the oracle's decode on whole (batch, kv-head) units of the same
+    workload.  Returns (KV tokens/s, threads used, description)."""
+    from oracle import tq_oracle as O
+    g = w.q_heads // w.kv_heads
+    kcent = O.codebook_f32(w.k_bits)[0]
+    vcent = O.codebook_f32(w.v_bits)[0]
+    signs = O.sign_vector(w.sign_seed)
+    done_tok = 0.0
+    t_wall = 0.0
+    c0 = time.process_time()
+    done = []
+    for (b, h) in units:
+        sl = slice(h, h + 1)
+        t = time.perf_counter()
+        O.decode_rotated(w.q[b:b + 1, h * g:(h + 1) * g].astype(np.float64), kc[b:b + 1, sl],
+                         kn[b:b + 1, sl], vc[b:b + 1, sl], vn[b:b + 1, sl], w.seq_lens[b:b + 1],
+                         w.scale, w.k_bits, w.v_bits, kcent, vcent, signs, w.sparse_thr)
+        t_wall += time.perf_counter() - t
+        done_tok += float(w.seq_lens[b]) / w.kv_heads  # one kv-head of each position
+        done.append((b, h))
+        if t_wall > budget_s:
+            break
+    cpu = time.process_time() - c0
+    threads = max(1, int(round(cpu / max(t_wall, 1e-9))))
+    desc = (f"oracle decode (fp64, formulation B) of {len(done)} (batch, kv-head) unit(s) "
+            f"{done} of this workload, {int(sum(w.seq_lens[b] for b, _ in done))} positions x "
+            f"{g} q-heads; KV tokens counted as positions / kv_heads")
+    return done_tok / t_wall, threads, desc
+
+
+# ------------------------------------------------------------- traffic --
+
+def recorded_traffic(kernel_file, name):
+    """dram bytes per launch from a committed ncu summary, only if the kernel
+    source is unchanged since the capture (sha256 recorded beside it)."""
+    path = os.path.join(ROOT, "profiles", name)
+    src = os.path.join(ROOT, "quantized_decode_attention_tq_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if fields.get("kernel_sha256") != sha or "dram_bytes_per_launch" not in fields:
+        return None
+    return float(fields["dram_bytes_per_launch"])
+
+
+# ------------------------------------------------------------- main arms --
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import tq_oracle as O
+    w = workload(args.workload)
+    # the oracle encodes the sampled unit itself (it may not use GPU results)
+    g = w.q_heads // w.kv_heads
+    kcent, kt = O.codebook_f32(w.k_bits)
+    vcent, vt = O.codebook_f32(w.v_bits)
+    s = O.sign_vector(w.sign_seed)
+    b, h = 0, 0
+    kc, kn, _ = O.encode(w.k[b:b + 1, h:h + 1], s, w.k_bits, kt)
+    vc, vn, _ = O.encode(w.v[b:b + 1, h:h + 1], s, w.v_bits, vt)
+    times = []
+    c0 = time.process_time()
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        O.decode_rotated(w.q[b:b + 1, h * g:(h + 1) * g].astype(np.float64), kc, kn, vc, vn,
+                         w.seq_lens[b:b + 1], w.scale, w.k_bits, w.v_bits, kcent, vcent, s, w.sparse_thr)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+        if sum(times) > 120:
+            break
+    wall = sum(times)
+    threads = max(1, int(round((time.process_time() - c0) / max(wall + 1e-9, 1e-9))))
+    toks = float(w.seq_lens[b]) / w.kv_heads
+    value = toks * len(times) / wall
+    sample = (f"oracle decode (fp64) of unit (batch 0, kv-head 0): {int(w.seq_lens[b])} positions x {g} "
+              f"q-heads per step, {len(times)} steps; KV tokens counted as positions / kv_heads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "KV tokens/s",
+            "n_gpus": args.gpus, "steps": len(times), "warmup": args.warmup,
+            "ms_per_step": 1e3 * wall / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[args.workload]},
+            "cpu_baseline": {"value": value, "unit": "KV tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "KV tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_tq(args):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_decode_attention_tq_b200 as tq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def allmax(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def allsum(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    w = workload(args.workload, rank)
+    desc = tq.kv_desc(w.batch, w.kv_heads, w.head_dim, w.seq_cap, w.k_bits, w.v_bits, w.sign_seed)
+    kcb, vcb = tq.make_codebook(w.k_bits), tq.make_codebook(w.v_bits)
+
+    # ---- build the packed cache with the library's encoder, then copies ----
+    cache0 = tq.alloc_cache(desc, dev)
+    tq.encode_kv(cache0, kcb, vcb, torch.from_numpy(w.k).to(dev), torch.from_numpy(w.v).to(dev))
+    torch.cuda.synchronize()
+    kvb = kv_bytes(w)
+    cache_bytes = sum(t.numel() * t.element_size() for t in
+                      (cache0.k_codes, cache0.k_norms, cache0.v_codes, cache0.v_norms))
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_copies = max(2, math.ceil(3 * l2 / max(cache_bytes, 1)) + 1)
+    caches = [cache0] + [tq.Cache(desc, cache0.k_codes.clone(), cache0.k_norms.clone(),
+                                  cache0.v_codes.clone(), cache0.v_norms.clone())
+                         for _ in range(n_copies - 1)]
+
+    # step inputs: the newest row of every (batch, kv-head) and the query
+    lens_np = w.seq_lens.astype(np.int32)
+    pos_np = (lens_np - 1).astype(np.int32)
+    k_new_np = np.ascontiguousarray(w.k[np.arange(w.batch), :, pos_np][:, :, None, :])
+    v_new_np = np.ascontiguousarray(w.v[np.arange(w.batch), :, pos_np][:, :, None, :])
+    q = torch.from_numpy(w.q).to(dev)
+    k_new = torch.from_numpy(k_new_np).to(dev)
+    v_new = torch.from_numpy(v_new_np).to(dev)
+    lens = torch.from_numpy(lens_np).to(dev)
+    start = torch.from_numpy(pos_np).to(dev)
+    out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float32, device=dev)
+    ws = tq.alloc_workspace(desc, w.q_heads, w.sparse_thr, dev)
+    decode_launches = 2 if w.sparse_thr > 0 else 1
+
+    def enc(c):
+        tq.encode_kv(caches[c], kcb, vcb, k_new, v_new, start_pos=start)
+
+    def dec(c):
+        tq.decode_attention(caches[c], kcb, vcb, q, lens, w.scale, out, ws, sparse_thr=w.sparse_thr)
+
+    for c in range(n_copies):  # eager warm-up (also primes the launch caches)
+        enc(c)
+        dec(c)
+    torch.cuda.synchronize()
+
+    # ---- CUDA graphs: one for the encode launch, one for the decode launch(es)
+    g_enc, g_dec = [], []
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for c in range(n_copies):
+            ge, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ge, stream=s):
+                enc(c)
+            with torch.cuda.graph(gd, stream=s):
+                dec(c)
+            g_enc.append(ge)
+            g_dec.append(gd)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        g_enc[i % n_copies].replay()
+        g_dec[i % n_copies].replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region -------------------------------------------------------
+    stream = torch.cuda.current_stream()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ea = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    eb = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    ev0.record(stream)
+    for i in range(args.steps):
+        c = i % n_copies
+        g_enc[c].replay()
+        ea[i].record(stream)
+        g_dec[c].replay()
+        eb[i].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier()
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    dec_ms_local = statistics.mean(a.elapsed_time(b) for a, b in zip(ea, eb))
+    ms = allmax(ms_local)
+    dec_ms = allmax(dec_ms_local)
+    tokens_step = allsum(float(np.sum(w.seq_lens)))
+    value = tokens_step / (ms / 1e3)
+
+    # ---- end to end through the public API with host buffers ---------------
+    h2d, d2h = step_io_bytes(w)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    q_h, k_h, v_h, l_h, s_h = pin(w.q), pin(k_new_np), pin(v_new_np), pin(lens_np), pin(pos_np)
+    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+
+    def e2e_step(c):
+        q.copy_(q_h, non_blocking=True)
+        k_new.copy_(k_h, non_blocking=True)
+        v_new.copy_(v_h, non_blocking=True)
+        lens.copy_(l_h, non_blocking=True)
+        start.copy_(s_h, non_blocking=True)
+        enc(c)
+        dec(c)
+        out_h.copy_(out, non_blocking=True)
+
+    for i in range(max(3, args.warmup)):
+        e2e_step(i % n_copies)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i % n_copies)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allmax(e0.elapsed_time(e1) / args.steps)
+    e2e_value = tokens_step / (e2e_ms / 1e3)
+
+    # ---- encoder alone on the encode-only workload -------------------------
+    encode_info = None
+    if not args.no_encode and rank == 0:
+        from quantized_decode_attention_tq_b200 import inputs
+        del caches, g_enc, g_dec
+        torch.cuda.empty_cache()
+        we = inputs.make("encode", with_q=False)
+        de = tq.kv_desc(we.batch, we.kv_heads, we.head_dim, we.seq_cap, we.k_bits, we.v_bits)
+        ce = tq.alloc_cache(de, dev)
+        ke, ve = torch.from_numpy(we.k).to(dev), torch.from_numpy(we.v).to(dev)
+        kcb_e, vcb_e = tq.make_codebook(we.k_bits), tq.make_codebook(we.v_bits)
+        for _ in range(3):
+            tq.encode_kv(ce, kcb_e, vcb_e, ke, ve)
+        torch.cuda.synchronize()
+        n_enc = 20
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(n_enc):
+            tq.encode_kv(ce, kcb_e, vcb_e, ke, ve)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        enc_ms = x0.elapsed_time(x1) / n_enc
+        n_blocks = we.batch * we.kv_heads * we.seq_cap
+        enc_bytes = ke.numel() * 2 * 2 + n_blocks * ((16 * we.k_bits + 2) + (16 * we.v_bits + 2))
+        peak, _ = measured_peaks()
+        encode_info = {"workload": "encode-only B8 Hkv8 D128 S32768 fp16 in, K3 (outlier-scaled "
+                                   "Gaussian) / V2 (Student-t4)",
+                       "gbs": enc_bytes / (enc_ms / 1e3) / 1e9, "us": enc_ms * 1e3,
+                       "bytes": enc_bytes, "frac_of_measured_hbm": enc_bytes / (enc_ms / 1e3) / 1e9 / peak,
+                       "l2": "1.25 GB streamed per launch (> L2)"}
+
+    # ---- CPU oracle baseline (rank 0, N = 1) --------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        kc = cache0.k_codes.cpu().numpy()
+        kn = cache0.k_norms.cpu().numpy().view(np.float16)
+        vc = cache0.v_codes.cpu().numpy()
+        vn = cache0.v_norms.cpu().numpy().view(np.float16)
+        units = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+        v_cpu, threads, sample = cpu_oracle_sample(w, kc, kn, vc, vn, units, budget_s=15.0)
+        cpu = {"value": v_cpu, "unit": "KV tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        achieved = kvb / (dec_ms / 1e3) / 1e9
+        traffic = recorded_traffic("tq_decode.cu", f"decode_{args.workload}_traffic.txt")
+        line = {
+            "metric": METRIC, "value": value, "unit": "KV tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16xf16->f32 (tensor-core products of fp16 codewords, fp32 softmax/accumulate)",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAMES[args.workload], "batch_per_gpu": w.batch,
+                       "seq_len": w.seq_cap, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                       "head_dim": w.head_dim, "k_bits": w.k_bits, "v_bits": w.v_bits,
+                       "sparse_thr": w.sparse_thr, "parallelism": f"independent batches x{world}",
+                       "l2": f"rotating {n_copies} cache copies of {cache_bytes / 1e6:.0f} MB (> 3x L2)"},
+            "decode_us": dec_ms * 1e3, "hbm_gbs": achieved,
+            "hbm_frac_of_8tbs": achieved / 8000.0,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": kvb},
+            "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * (1 + decode_launches),
+            "clocks": clocks,
+            "encode": encode_info,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_tq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * tq.h -- C ABI of a TurboQuant-style compressed KV cache for one NVIDIA B200
+ * (sm_100a): an encoder that writes packed b-bit codes plus one fp16 norm per
+ * 128-element block, and single-token decode attention that reads the packed
+ * cache directly.
+ *
+ * Method (pages cited by title and section):
+ *   - "TheTom/llama-cpp-turboquant" README, table "量化类型": every turbo KV
+ *     format rotates 128-element blocks with a Walsh-Hadamard transform and
+ *     then quantises them with a (polar: radius + direction) codebook.
+ *   - intelliparadigm TurboQuant article, §3.2: the rotation is a randomized
+ *     Hadamard transform, a Hadamard matrix combined with a random +-1
+ *     diagonal, computed with the O(d log d) fast transform; §3.3: the scalar
+ *     quantiser is Lloyd-Max.
+ *   - "llama-tq" article, section on the K cache: Q.K is evaluated in the
+ *     Hadamard domain so the K cache is never dequantised.
+ *   - README "压缩策略" and "TurboQuant+" section "注意力门控稀疏V解压": V
+ *     positions whose softmax weight is below a threshold are skipped and
+ *     count as zero.
+ *
+ * Conventions that hold for every entry point:
+ *   - Ownership: the caller allocates and owns every buffer.  The library
+ *     never allocates device memory and keeps no pointer after a call returns.
+ *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *     default stream).  Device work is asynchronous on that stream; only
+ *     tq_make_codebook and tq_sign_vector are synchronous (host only).
+ *   - Errors: every call returns a tq_status code and never throws.  Host-side
+ *     validation runs first; when it fails nothing is launched.  Range errors
+ *     that only the device can see (a position or a length outside the cache,
+ *     an fp16 norm overflow) set bits of the caller's optional device status
+ *     word (`dev_status`, one uint32 in device memory, may be NULL); the
+ *     offending rows are clamped or skipped and the kernel never traps.
+ *   - Block layout: D = head_dim is a multiple of 128; nb = D / 128 blocks
+ *     per vector.  For b-bit codes one block stores 16*b bytes of codes
+ *     (index i of the block at stream bits [b*i, b*i+b), LSB-first,
+ *     little-endian bytes) and one fp16 norm: b + 16/128 bits per value.
+ *   - Cache tensors (row-major, contiguous):
+ *       codes [batch, kv_heads, seq_cap, nb, 16*b]  uint8
+ *       norms [batch, kv_heads, seq_cap, nb]        fp16 (stored as uint16)
+ *     K and V are separate tensors, each with its own bit width.  Code
+ *     tensors must be 16-byte aligned, norm tensors 4-byte aligned.
+ *   - GQA: q-head h reads kv-head h / (q_heads / kv_heads).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ_BLOCK 128
+
+/* Return codes. */
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment           */
+  TQ_ERR_UNSUPPORTED = 2,  /* valid but not built: bits, head_dim, group     */
+  TQ_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required     */
+  TQ_ERR_CUDA = 4          /* a CUDA runtime call failed (launch, attribute) */
+} tq_status;
+
+/* Bits of the device status word (sticky; the library only ORs into it). */
+#define TQ_DEV_POS_RANGE 1u      /* encode row outside [0, seq_cap): skipped */
+#define TQ_DEV_NORM_OVERFLOW 2u  /* block norm above fp16 max: saturated     */
+#define TQ_DEV_LEN_RANGE 4u      /* seq_lens[b] outside [0, seq_cap]: clamped */
+
+typedef enum { TQ_F32 = 0, TQ_F16 = 1 } tq_dtype;
+
+/* Lloyd-Max codebook for N(0,1) with L = 2^bits levels: centroids[0..L-1]
+ * ascending and symmetric, boundaries[0..L-2] the midpoints.  Unused tail
+ * entries are zero. */
+typedef struct {
+  int32_t bits;
+  float centroids[16];
+  float boundaries[15];
+} tq_codebook;
+
+/* Shape and format of one layer's compressed KV cache. */
+typedef struct {
+  int32_t batch;     /* B >= 1                                   */
+  int32_t kv_heads;  /* Hkv >= 1                                 */
+  int32_t head_dim;  /* D, a multiple of 128: encode <= 512, decode <= 256 */
+  int32_t seq_cap;   /* S_cap >= 1: positions per (b, kv-head)   */
+  uint64_t sign_seed;/* seed of the +-1 diagonal (SplitMix64)    */
+  int32_t k_bits;    /* 2, 3 or 4                                */
+  int32_t v_bits;    /* 2, 3 or 4                                */
+} tq_kv_desc;
+
+/*
+ * tq_make_codebook -- Lloyd-Max quantiser of the standard normal density.
+ * Source: intelliparadigm TurboQuant article §3.3 (initialise centres, assign
+ * each point to the nearest centre, move each centre to the mean of its
+ * points, repeat to convergence), run on the N(0,1) density itself.
+ * bits: 1..4.  out: host pointer.  Synchronous, host only, no CUDA calls.
+ * Returns TQ_ERR_INVALID_ARG for a null `out`, TQ_ERR_UNSUPPORTED for bits
+ * outside 1..4.
+ */
+int tq_make_codebook(int bits, tq_codebook* out);
+
+/*
+ * tq_sign_vector -- the 128 entries (+1 or -1) of the random diagonal D of
+ * the rotation H.D (intelliparadigm TurboQuant article §3.2).  Entry i is -1
+ * when the top bit of the i-th SplitMix64 output from state `seed` is set.
+ * out: host array of 128 int8.  Synchronous, host only.
+ */
+int tq_sign_vector(uint64_t seed, int8_t* out);
+
+/*
+ * tq_encode_kv -- write `seq_new` new positions of K and V into the cache.
+ * Per 128-element block ("TheTom/llama-cpp-turboquant" README table
+ * "量化类型"; TurboQuant article §3.2-§3.3): x_s = s o x; y = H.x_s (fast
+ * WHT, unnormalised); n = ||x||_2 stored as fp16 (round to nearest even);
+ * idx_i = #{ j : boundaries[j] < y_i / n }; idx bit-packed as described above.
+ *
+ * k, v: device, [batch, kv_heads, seq_new, head_dim] contiguous, dtype
+ *       in_dtype (TQ_F32 or TQ_F16), 16-byte aligned.  Either may be NULL to
+ *       encode only the other side (its codes/norms pointers may then be NULL).
+ * start_pos: device int32 [batch] (row t of batch b goes to position
+ *       start_pos[b] + t) or NULL (= 0).  Rows that would land outside
+ *       [0, seq_cap) are skipped and set TQ_DEV_POS_RANGE.
+ * k_cb, v_cb: host codebooks whose bits equal desc->k_bits / desc->v_bits.
+ * dev_status: optional device uint32 (see above).
+ * seq_new == 0 is a no-op.  Returns TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED
+ * on bad arguments (nothing launched), TQ_ERR_CUDA if the launch fails.
+ */
+int tq_encode_kv(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                 const void* k, const void* v, int in_dtype, int seq_new,
+                 const int32_t* start_pos, uint8_t* k_codes, uint16_t* k_norms,
+                 uint8_t* v_codes, uint16_t* v_norms, uint32_t* dev_status, void* stream);
+
+/*
+ * tq_decode_workspace_size -- bytes of device workspace tq_decode_attention
+ * needs for this cache shape, q_heads and sparse setting (sparse_thr > 0 adds
+ * an fp32 score buffer of batch * q_heads * seq_cap entries).  Returns 0 for
+ * invalid arguments.
+ */
+size_t tq_decode_workspace_size(const tq_kv_desc* desc, int q_heads, float sparse_thr);
+
+/*
+ * tq_decode_attention -- one query token per sequence against the packed
+ * cache ("llama-tq" article, K-cache section: Q.K in the Hadamard domain, no
+ * K dequantisation; README "压缩策略": sparse-V).
+ *   q^ = H.(s o q) per block, once per q-head;
+ *   s_t = scale * sum_blk (nK_t,blk / 128) * q^_blk . cK[idx_t,blk];
+ *   w = softmax over t < seq_lens[b];
+ *   o = sum_t w_t vt_t, computed as s o (H.acc) with
+ *       acc = sum_t w_t (nV_t,blk / 128) cV[idx_t,blk] (V summed in the
+ *       rotated domain, one inverse rotation per head).
+ * Sparse-V (sparse_thr > 0): positions with w_t < sparse_thr (w the
+ * normalised weight) contribute zero and the rest are not renormalised.
+ *
+ * Supported: head_dim 128 or 256 (TQ_ERR_UNSUPPORTED otherwise), batch <=
+ * 4096, any q_heads / kv_heads ratio (groups above 8 run in slices of 8).
+ * q: device [batch, q_heads, head_dim], q_dtype TQ_F32 or TQ_F16.
+ *    q_heads must be a multiple of kv_heads.
+ * seq_lens: device int32 [batch]; values are clamped to [0, seq_cap]
+ *    (TQ_DEV_LEN_RANGE).  A length of 0 gives an all-zero output row.
+ * out: device fp32 [batch, q_heads, head_dim].
+ * workspace: device buffer of at least tq_decode_workspace_size() bytes,
+ *    256-byte aligned.  It must be all-zero before its first use; every call
+ *    that runs to completion leaves it ready for the next call.  Calls that
+ *    share one workspace must not overlap in time (use one stream).
+ * Returns TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED / TQ_ERR_WORKSPACE on bad
+ * arguments (nothing launched), TQ_ERR_CUDA if a launch fails.
+ */
+int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                        int q_heads, const void* q, int q_dtype,
+                        const uint8_t* k_codes, const uint16_t* k_norms,
+                        const uint8_t* v_codes, const uint16_t* v_norms,
+                        const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                        void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                        void* stream);
+
+/* Static description of a status code. */
+const char* tq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H_ */

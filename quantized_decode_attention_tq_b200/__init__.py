@@ -1,0 +1,17 @@
+"""TurboQuant-style compressed KV cache for NVIDIA B200 (sm_100a).
+
+The compute lives in the C-ABI library ``libtq_b200.so`` (include/tq.h);
+this package is its thin Python binding plus the seeded synthetic workloads.
+"""
+from ._lib import (TQ_DEV_LEN_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_POS_RANGE, TQ_F16, TQ_F32,
+                   Codebook, KVDesc, TQError, lib)
+from .api import (Cache, alloc_cache, alloc_workspace, cache_shapes, codebook_arrays,
+                  decode_attention, decode_workspace_size, encode_kv, kv_desc, make_codebook,
+                  sign_vector)
+
+__all__ = [
+    "Cache", "Codebook", "KVDesc", "TQError", "TQ_F16", "TQ_F32", "TQ_DEV_LEN_RANGE",
+    "TQ_DEV_NORM_OVERFLOW", "TQ_DEV_POS_RANGE", "alloc_cache", "alloc_workspace", "cache_shapes",
+    "codebook_arrays", "decode_attention", "decode_workspace_size", "encode_kv", "kv_desc",
+    "lib", "make_codebook", "sign_vector",
+]

@@ -1,0 +1,138 @@
+"""Thin Python binding over the C ABI (include/tq.h).
+
+Argument marshalling only: torch tensors supply device memory and the current
+CUDA stream; every step of the encoder and of decode attention runs in the
+library's sm_100a kernels.  There is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+
+from ._lib import (TQ_F16, TQ_F32, Codebook, KVDesc, check, lib)
+
+
+def make_codebook(bits: int) -> Codebook:
+    """Lloyd-Max codebook of N(0,1) with 2^bits levels (host, synchronous)."""
+    cb = Codebook()
+    check("tq_make_codebook", lib().tq_make_codebook(bits, ctypes.byref(cb)))
+    return cb
+
+
+def codebook_arrays(cb: Codebook):
+    levels = 1 << cb.bits
+    return (np.array(cb.centroids[:levels], dtype=np.float32),
+            np.array(cb.boundaries[:levels - 1], dtype=np.float32))
+
+
+def sign_vector(seed: int) -> np.ndarray:
+    out = (ctypes.c_int8 * 128)()
+    check("tq_sign_vector", lib().tq_sign_vector(seed, out))
+    return np.frombuffer(out, dtype=np.int8).copy()
+
+
+def kv_desc(batch, kv_heads, head_dim, seq_cap, k_bits, v_bits, sign_seed=0) -> KVDesc:
+    return KVDesc(batch, kv_heads, head_dim, seq_cap, sign_seed, k_bits, v_bits)
+
+
+@dataclass
+class Cache:
+    """One layer's packed cache: codes uint8, norms fp16 stored in int16 tensors."""
+    desc: KVDesc
+    k_codes: "object"
+    k_norms: "object"
+    v_codes: "object"
+    v_norms: "object"
+
+
+def cache_shapes(desc: KVDesc):
+    nb = desc.head_dim // 128
+    base = (desc.batch, desc.kv_heads, desc.seq_cap, nb)
+    return {"k_codes": base + (16 * desc.k_bits,), "k_norms": base,
+            "v_codes": base + (16 * desc.v_bits,), "v_norms": base}
+
+
+def alloc_cache(desc: KVDesc, device="cuda") -> Cache:
+    import torch
+    s = cache_shapes(desc)
+    return Cache(desc,
+                 torch.zeros(s["k_codes"], dtype=torch.uint8, device=device),
+                 torch.zeros(s["k_norms"], dtype=torch.int16, device=device),
+                 torch.zeros(s["v_codes"], dtype=torch.uint8, device=device),
+                 torch.zeros(s["v_norms"], dtype=torch.int16, device=device))
+
+
+def _ptr(t, name):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float16:
+        return TQ_F16
+    if t.dtype == torch.float32:
+        return TQ_F32
+    raise ValueError(f"unsupported dtype {t.dtype}: fp16 or fp32")
+
+
+def encode_kv(cache: Cache, k_cb: Codebook, v_cb: Codebook, k=None, v=None, start_pos=None,
+              status=None, stream=None) -> None:
+    """Encode K/V rows [B, Hkv, seq_new, D] into the cache (tq_encode_kv)."""
+    src = k if k is not None else v
+    if src is None:
+        raise ValueError("k or v is required")
+    if k is not None and v is not None and (k.shape != v.shape or k.dtype != v.dtype):
+        raise ValueError("k and v must have the same shape and dtype")
+    seq_new = src.shape[2]
+    st = lib().tq_encode_kv(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb),
+        _ptr(k, "k"), _ptr(v, "v"), _dtype_code(src), seq_new, _ptr(start_pos, "start_pos"),
+        _ptr(cache.k_codes, "k_codes") if k is not None else None,
+        _ptr(cache.k_norms, "k_norms") if k is not None else None,
+        _ptr(cache.v_codes, "v_codes") if v is not None else None,
+        _ptr(cache.v_norms, "v_norms") if v is not None else None,
+        _ptr(status, "status"), _stream(stream))
+    check("tq_encode_kv", st)
+
+
+def decode_workspace_size(desc: KVDesc, q_heads: int, sparse_thr: float = 0.0) -> int:
+    return int(lib().tq_decode_workspace_size(ctypes.byref(desc), q_heads, sparse_thr))
+
+
+def alloc_workspace(desc: KVDesc, q_heads: int, sparse_thr: float = 0.0, device="cuda"):
+    """A zeroed workspace (the library requires zero before first use)."""
+    import torch
+    n = decode_workspace_size(desc, q_heads, sparse_thr)
+    if n == 0:
+        raise ValueError("invalid decode configuration")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def decode_attention(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, scale: float,
+                     out, workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """Single-token decode attention over the packed cache (tq_decode_attention)."""
+    q_heads = q.shape[1]
+    st = lib().tq_decode_attention(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb), q_heads,
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention", st)
+    return out

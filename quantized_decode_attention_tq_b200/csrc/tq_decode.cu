@@ -1,0 +1,804 @@
+// Decode attention over the packed TurboQuant cache (one query token per
+// sequence, GQA, per-sequence lengths, optional exact sparse-V).
+//
+// Method: "llama-tq" article, K-cache section (Q.K in the Hadamard domain,
+// no K dequantisation); "TheTom/llama-cpp-turboquant" README, table "量化类型"
+// (WHT + codebook on 128-element blocks) and "压缩策略" (sparse-V dequant);
+// "TurboQuant+" section "注意力门控稀疏V解压" (skipped V counts as zero).
+//
+// Kernel design (sm_100a):
+//  * Work = (unit, 16-token tile), unit = (batch, kv-head, group of <= 8
+//    q-heads).  All tiles of all units are laid end to end and cut into
+//    gridDim.x equal ranges, one per persistent CTA (stream-K style), so
+//    ragged lengths balance to within one tile.  A CTA writes one partial
+//    (m, l, acc) per unit it touches; the CTA that completes a unit (atomic
+//    tile count) merges the partials in a fixed order and applies the inverse
+//    rotation, so results do not depend on scheduling.
+//  * Scores: S[16 tok x 8 heads] = Kc[16 x 128] . Qhat[128 x 8] with
+//    mma.sync m16n8k16 (f16 in, f32 accumulate).  K codes are turned into f16
+//    A fragments in registers through a shared-memory table indexed by two
+//    codes and replicated per lane (conflict-free).  Contraction order is
+//    permuted so each lane's fragment comes from 32 contiguous codes.
+//  * Online softmax in the log2 domain with a lazy rescale (only when the
+//    running max grows by more than 2^6), exact because the stored max is the
+//    one every exponent used.
+//  * P.V: O^T[128 dims x 8 heads] += Vc^T[dims x 16 tok] . P'^T[16 tok x 8],
+//    P' = p * nV / 128; the score accumulator becomes the B fragment with two
+//    movmatrix transposes.  V stays in the rotated domain until the end.
+//  * Sparse-V is exact and two-pass: pass 1 stores log2-domain scores and
+//    per-partial (m, l); pass 2 forms the log-sum-exp, zeroes the normalised
+//    weights below the threshold and accumulates V with the rest.
+
+#include <cuda_fp16.h>
+
+#include "../../include/tq.h"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr float kTau = 6.0f;        // lazy-rescale threshold (log2 units)
+constexpr int kPrefetchDist = 2;    // L2 bulk prefetch, in warp-loop steps
+
+enum Mode { kFused = 0, kScores = 1, kSparseV = 2 };
+
+// ----------------------------------------------------------------- helpers --
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t movtrans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  return __byte_perm(a, b, sel);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Byte offset into a lane-replicated table: field of `fb` bits at bit `pos`
+// of the word array w, times 128 (32 lanes x 4 bytes per entry), plus lane*4.
+// Called with compile-time pos/fb after unrolling, so the branches fold.
+__device__ __forceinline__ uint32_t lut_off(const uint32_t* w, int pos, int fb, uint32_t lane4) {
+  const int wi = pos >> 5, sh = pos & 31;
+  const uint32_t mask = ((1u << fb) - 1u) << 7;
+  uint32_t v;
+  if (sh + fb <= 32)
+    v = (sh >= 7) ? (w[wi] >> (sh - 7)) : (w[wi] << (7 - sh));
+  else
+    v = __funnelshift_r(w[wi], w[wi + 1], sh) << 7;
+  return (v & mask) | lane4;
+}
+
+__device__ __forceinline__ uint32_t lds(const uint8_t* base, uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(base + off);
+}
+
+template <int B>
+struct Fmt {
+  static constexpr int kEntries = 1 << (2 * B);
+  static constexpr int kLutBytes = kEntries * 128;
+  static constexpr int kBlockBytes = 16 * B;
+};
+
+// Registers holding one 16-token tile for one lane.
+// Lane (R = lane/4, g = lane%4):
+//   K rows: tokens R and R+8, codes of dims [32g, 32g+32) of each block;
+//   V cols: tokens 2g, 2g+1, 2g+8, 2g+9, codes of dims [16R, 16R+16);
+//   norms : tokens R and R+8.
+template <int KB, int VB, int NB>
+struct TileRegs {
+  uint32_t k[2][NB][KB > 0 ? KB : 1];
+  uint32_t v[4][NB][2];
+  float kn[2][NB];
+  float vn[2][NB];
+};
+
+struct UnitPtrs {
+  const uint8_t* kc;
+  const uint16_t* kn;
+  const uint8_t* vc;
+  const uint16_t* vn;
+  int len;
+};
+
+template <int KB, int VB, int NB, bool LOADK, bool LOADV>
+__device__ __forceinline__ void load_tile(TileRegs<KB, VB, NB>& r, const UnitPtrs& u, int t0,
+                                          int lane) {
+  const int R = lane >> 2, g = lane & 3;
+  if constexpr (LOADK) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int t = t0 + R + 8 * rr;
+      const bool ok = t < u.len;
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        const uint8_t* src = u.kc + ((size_t)t * NB + blk) * Fmt<KB>::kBlockBytes + g * KB * 4;
+        if constexpr (KB == 4) {
+          uint4 x = ok ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
+          r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y; r.k[rr][blk][2] = x.z; r.k[rr][blk][3] = x.w;
+        } else if constexpr (KB == 3) {
+          const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
+          r.k[rr][blk][0] = ok ? __ldg(s) : 0u;
+          r.k[rr][blk][1] = ok ? __ldg(s + 1) : 0u;
+          r.k[rr][blk][2] = ok ? __ldg(s + 2) : 0u;
+        } else {
+          uint2 x = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0, 0);
+          r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y;
+        }
+        r.kn[rr][blk] = ok ? __half2float(__ushort_as_half(__ldg(u.kn + (size_t)t * NB + blk))) : 0.0f;
+      }
+    }
+  }
+  if constexpr (LOADV) {
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+      const int t = t0 + 2 * g + (tt & 1) + 8 * (tt >> 1);
+      const bool ok = t < u.len;
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        const uint8_t* blkp = u.vc + ((size_t)t * NB + blk) * Fmt<VB>::kBlockBytes;
+        if constexpr (VB == 4) {
+          uint2 x = ok ? __ldg(reinterpret_cast<const uint2*>(blkp + 8 * R)) : make_uint2(0, 0);
+          r.v[tt][blk][0] = x.x; r.v[tt][blk][1] = x.y;
+        } else if constexpr (VB == 3) {
+          // 6 bytes at byte 6R: covered by 32-bit words (3R)/2 and (3R)/2 + 1.
+          const uint32_t* s = reinterpret_cast<const uint32_t*>(blkp) + ((3 * R) >> 1);
+          uint32_t w0 = ok ? __ldg(s) : 0u, w1 = ok ? __ldg(s + 1) : 0u;
+          if (R & 1) { w0 = __funnelshift_r(w0, w1, 16); w1 >>= 16; }
+          r.v[tt][blk][0] = w0; r.v[tt][blk][1] = w1;
+        } else {
+          r.v[tt][blk][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(blkp) + R) : 0u;
+          r.v[tt][blk][1] = 0u;
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int t = t0 + R + 8 * rr;
+      const bool ok = t < u.len;
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk)
+        r.vn[rr][blk] = ok ? __half2float(__ushort_as_half(__ldg(u.vn + (size_t)t * NB + blk))) * (1.0f / kBlock) : 0.0f;
+    }
+  }
+}
+
+// Issue L2 prefetches for one future tile (one lane per warp).
+template <int KB, int VB, int NB, bool PK, bool PV>
+__device__ __forceinline__ void prefetch_tile(const UnitPtrs& u, int t0, int seq_cap) {
+  const int n = min(kTile, seq_cap - t0);
+  if (n <= 0) return;
+  if constexpr (PK) prefetch_l2(u.kc + (size_t)t0 * NB * Fmt<KB>::kBlockBytes, n * NB * Fmt<KB>::kBlockBytes);
+  if constexpr (PV) prefetch_l2(u.vc + (size_t)t0 * NB * Fmt<VB>::kBlockBytes, n * NB * Fmt<VB>::kBlockBytes);
+}
+
+// ----------------------------------------------------- shared-memory plan --
+
+template <int KB, int VB, int NB, int MODE>
+struct Smem {
+  static constexpr int D = NB * kBlock;
+  static constexpr bool kHasK = MODE != kSparseV;
+  static constexpr bool kHasV = MODE != kScores;
+  static constexpr int kLutK = kHasK ? Fmt<KB>::kLutBytes : 0;
+  static constexpr int kLutV = kHasV ? Fmt<VB>::kLutBytes : 0;
+  static constexpr int kWorkFloats = kWarps * kMaxGroup * D;     // per-warp partials / qhat
+  static constexpr int kResFloats = kMaxGroup * D;               // merged rotated-domain acc
+  static constexpr int kOffLutK = 0;
+  static constexpr int kOffLutV = kOffLutK + kLutK;
+  static constexpr int kOffWork = kOffLutV + kLutV;
+  static constexpr int kOffRes = kOffWork + kWorkFloats * 4;
+  static constexpr int kOffMisc = kOffRes + kResFloats * 4;
+  // misc: warp m/l [kWarps][8] x2, merged M/L/lse [8] x3, qexp [8], flag, then batch prefix.
+  static constexpr int kMiscFloats = 2 * kWarps * kMaxGroup + 4 * kMaxGroup + 4;
+  static constexpr int kOffPrefix = kOffMisc + kMiscFloats * 4;
+  static size_t bytes(int batch) { return (size_t)kOffPrefix + (size_t)(batch + 1) * 4; }
+};
+
+// --------------------------------------------------------------- the kernel --
+
+template <int KB, int VB, int NB, int MODE>
+__global__ void __launch_bounds__(kThreads)
+decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
+  using SM = Smem<KB, VB, NB, MODE>;
+  constexpr int D = SM::D;
+  constexpr bool HASK = SM::kHasK, HASV = SM::kHasV;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* lutK = smem + SM::kOffLutK;
+  uint8_t* lutV = smem + SM::kOffLutV;
+  float* work = reinterpret_cast<float*>(smem + SM::kOffWork);
+  float* res = reinterpret_cast<float*>(smem + SM::kOffRes);
+  float* misc = reinterpret_cast<float*>(smem + SM::kOffMisc);
+  float* w_m = misc;                                  // [kWarps][8]
+  float* w_l = misc + kWarps * kMaxGroup;             // [kWarps][8]
+  float* u_M = misc + 2 * kWarps * kMaxGroup;         // [8]
+  float* u_L = u_M + kMaxGroup;                       // [8]
+  float* u_lse = u_L + kMaxGroup;                     // [8]
+  int* qexp = reinterpret_cast<int*>(u_lse + kMaxGroup);  // [8]
+  int* flag = qexp + kMaxGroup;
+  int* prefix = reinterpret_cast<int*>(smem + SM::kOffPrefix);  // [B+1] tiles per batch, prefix
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int R = lane >> 2, g = lane & 3;
+  const uint32_t lane4 = (uint32_t)lane * 4u;
+  const int G = p.q_heads / p.kv_heads;
+  const int n_hg = (G + kMaxGroup - 1) / kMaxGroup;
+  const int UB = p.kv_heads * n_hg;  // units per batch entry
+
+  // ---- tables: code pair -> half2 codewords, replicated for every lane ----
+  if constexpr (HASK) {
+    for (int e = tid; e < Fmt<KB>::kEntries * 32; e += kThreads) {
+      const int ent = e >> 5;
+      const float lo = p.kcent[ent & ((1 << KB) - 1)], hi = p.kcent[ent >> KB];
+      reinterpret_cast<uint32_t*>(lutK)[e] = pack_half2(lo, hi);
+    }
+  }
+  if constexpr (HASV) {
+    for (int e = tid; e < Fmt<VB>::kEntries * 32; e += kThreads) {
+      const int ent = e >> 5;
+      const float lo = p.vcent[ent & ((1 << VB) - 1)], hi = p.vcent[ent >> VB];
+      reinterpret_cast<uint32_t*>(lutV)[e] = pack_half2(lo, hi);
+    }
+  }
+
+  // ---- lengths: clamp, tiles per batch entry, exclusive prefix ------------
+  {
+    const int B = p.batch;
+    const int per = (B + kThreads - 1) / kThreads;
+    int local = 0;
+    const int b_lo = tid * per;
+    for (int b = b_lo; b < min(B, b_lo + per); ++b) {
+      int len = __ldg(p.seq_lens + b);
+      if (len < 0 || len > p.seq_cap) {
+        if (blockIdx.x == 0 && p.status) atomicOr(p.status, TQ_DEV_LEN_RANGE);
+        len = min(max(len, 0), p.seq_cap);
+      }
+      local += (len + kTile - 1) / kTile;
+    }
+    // block-wide exclusive scan of `local`
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) qexp[warp] = incl;  // temporary use of qexp as warp totals
+    __syncthreads();
+    int warp_off = 0;
+    for (int w = 0; w < warp; ++w) warp_off += qexp[w];
+    int run = warp_off + incl - local;
+    for (int b = b_lo; b < min(B, b_lo + per); ++b) {
+      prefix[b] = run;
+      int len = min(max(__ldg(p.seq_lens + b), 0), p.seq_cap);
+      run += (len + kTile - 1) / kTile;
+    }
+    if (tid == kThreads - 1) prefix[B] = run;
+    __syncthreads();
+  }
+  const long long T = (long long)prefix[p.batch] * UB;
+
+  // ---- zero rows of empty sequences (only the V-producing passes) ---------
+  if constexpr (MODE != kScores) {
+    const long long rows = (long long)p.batch * p.q_heads;
+    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+      const int b = (int)(row / p.q_heads);
+      if (prefix[b + 1] == prefix[b]) {
+        for (int d = tid; d < D; d += kThreads) p.out[row * D + d] = 0.0f;
+      }
+    }
+  }
+  if (T == 0) return;
+
+  const long long P = gridDim.x;
+  const long long lo = (long long)blockIdx.x * T / P;
+  const long long hi = ((long long)blockIdx.x + 1) * T / P;
+  auto cta_of = [&](long long x, long long parts) { return ((x + 1) * parts + T - 1) / T - 1; };
+
+  long long x = lo;
+  while (x < hi) {
+    // ---- locate the unit holding tile x ------------------------------------
+    const long long y = x / UB;  // in units of "tiles per batch entry"
+    int bl = 0, bh = p.batch;    // largest b with prefix[b] <= y
+    while (bh - bl > 1) {
+      const int mid = (bl + bh) >> 1;
+      if (prefix[mid] <= y) bl = mid; else bh = mid;
+    }
+    const int b = bl;
+    const int nt = prefix[b + 1] - prefix[b];
+    const long long TB = (long long)prefix[b] * UB;
+    const int r = (int)((x - TB) / nt);
+    const long long Su = TB + (long long)r * nt;
+    const int seg_lo = (int)(x - Su);
+    const int seg_hi = (int)(min(hi, Su + nt) - Su);
+    const int unit = b * UB + r;
+    const int kvh = r / n_hg, hg = r % n_hg;
+    const int h0 = kvh * G + hg * kMaxGroup;
+    const int Gu = min(kMaxGroup, G - hg * kMaxGroup);
+    const int len = min(max(__ldg(p.seq_lens + b), 0), p.seq_cap);
+
+    UnitPtrs up;
+    const size_t cache_row = (size_t)(b * p.kv_heads + kvh) * p.seq_cap;
+    up.kc = p.k_codes + cache_row * NB * Fmt<KB>::kBlockBytes;
+    up.kn = p.k_norms + cache_row * NB;
+    up.vc = p.v_codes + cache_row * NB * Fmt<VB>::kBlockBytes;
+    up.vn = p.v_norms + cache_row * NB;
+    up.len = len;
+
+    // ---- per-unit query preparation: qhat = H.(s o q) (D1) ----------------
+    uint32_t qf[NB][8][2];
+    float qmul[2];
+    float lse2[2] = {0.0f, 0.0f};
+    if constexpr (HASK) {
+      float* qs = work;  // [8][D]
+      for (int i = tid; i < kMaxGroup * D; i += kThreads) {
+        const int j = i / D, d = i % D;
+        float v = 0.0f;
+        if (j < Gu) {
+          const size_t qi = ((size_t)b * p.q_heads + h0 + j) * D + d;
+          v = p.q_f16 ? __half2float(reinterpret_cast<const __half*>(p.q)[qi])
+                      : reinterpret_cast<const float*>(p.q)[qi];
+          const int e = d & (kBlock - 1);
+          if ((p.sign_mask[e >> 5] >> (e & 31)) & 1u) v = -v;
+        }
+        qs[i] = v;
+      }
+      __syncthreads();
+      for (int s = 1; s < kBlock; s <<= 1) {
+        for (int i = tid; i < kMaxGroup * D / 2; i += kThreads) {
+          const int j = i / (D / 2), rem = i % (D / 2);
+          const int a = (rem / s) * 2 * s + (rem % s);
+          float* row = qs + j * D;
+          const float u = row[a], w = row[a + s];
+          row[a] = u + w;
+          row[a + s] = u - w;
+        }
+        __syncthreads();
+      }
+      // power-of-two scale per head so fp16 fragments neither overflow nor
+      // fall into subnormals
+      for (int j = warp; j < kMaxGroup; j += kWarps) {
+        float mx = 0.0f;
+        for (int d = lane; d < D; d += 32) mx = fmaxf(mx, fabsf(qs[j * D + d]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) qexp[j] = (mx > 0.0f) ? (ilogbf(mx) - 13) : 0;
+      }
+      __syncthreads();
+      const float qsc = ldexpf(1.0f, -qexp[R]);
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float* q4 = qs + R * D + blk * kBlock + 32 * g + 4 * j;
+          qf[blk][j][0] = pack_half2(q4[0] * qsc, q4[1] * qsc);
+          qf[blk][j][1] = pack_half2(q4[2] * qsc, q4[3] * qsc);
+        }
+      }
+      qmul[0] = p.score_mult * ldexpf(1.0f, qexp[2 * g]);
+      qmul[1] = p.score_mult * ldexpf(1.0f, qexp[2 * g + 1]);
+      __syncthreads();  // work area is reused below
+    }
+    if constexpr (MODE == kSparseV) {
+      // log-sum-exp (log2 domain) of every head of this unit, from the
+      // partials that pass 1 (p1_ctas CTAs) wrote
+      if (tid < Gu) {
+        const long long P1 = p1_ctas;
+        const long long c_first = cta_of(Su, P1), c_last = cta_of(Su + nt - 1, P1);
+        float M = -INFINITY;
+        for (long long c = c_first; c <= c_last; ++c) {
+          if (c * T / P1 == (c + 1) * T / P1) continue;  // empty range
+          M = fmaxf(M, __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2));
+        }
+        float L = 0.0f;
+        for (long long c = c_first; c <= c_last; ++c) {
+          if (c * T / P1 == (c + 1) * T / P1) continue;
+          const float* ml = p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2;
+          L += __ldcg(ml + 1) * ex2(__ldcg(ml) - M);
+        }
+        u_lse[tid] = M + __log2f(L);
+      }
+      __syncthreads();
+      lse2[0] = (2 * g < Gu) ? u_lse[2 * g] : 0.0f;
+      lse2[1] = (2 * g + 1 < Gu) ? u_lse[2 * g + 1] : 0.0f;
+    }
+    const float log2_thr = (MODE == kSparseV) ? __log2f(p.sparse_thr) : 0.0f;
+
+    // ---- warp loop over this segment's tiles ------------------------------
+    float acc[NB][8][4];
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[blk][mt][e] = 0.0f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.0f, 0.0f};
+
+    auto compute = [&](const TileRegs<KB, VB, NB>& tr, int tile) {
+      const int t0 = tile * kTile;
+      const bool okR = t0 + R < len, okR8 = t0 + R + 8 < len;
+      float pR[2], pR8[2];
+      if constexpr (HASK) {
+        // D2/D3: scores in the Hadamard domain, straight from the codes
+        float c[NB][4];
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk) {
+          c[blk][0] = c[blk][1] = c[blk][2] = c[blk][3] = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t a0 = lds(lutK, lut_off(tr.k[0][blk], 2 * KB * (2 * j), 2 * KB, lane4));
+            const uint32_t a1 = lds(lutK, lut_off(tr.k[1][blk], 2 * KB * (2 * j), 2 * KB, lane4));
+            const uint32_t a2 = lds(lutK, lut_off(tr.k[0][blk], 2 * KB * (2 * j + 1), 2 * KB, lane4));
+            const uint32_t a3 = lds(lutK, lut_off(tr.k[1][blk], 2 * KB * (2 * j + 1), 2 * KB, lane4));
+            mma16816(c[blk], a0, a1, a2, a3, qf[blk][j][0], qf[blk][j][1]);
+          }
+        }
+        float sR[2], sR8[2];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float a = 0.0f, bb = 0.0f;
+#pragma unroll
+          for (int blk = 0; blk < NB; ++blk) {
+            a = fmaf(c[blk][cc], tr.kn[0][blk], a);
+            bb = fmaf(c[blk][2 + cc], tr.kn[1][blk], bb);
+          }
+          sR[cc] = okR ? a * qmul[cc] : -INFINITY;
+          sR8[cc] = okR8 ? bb * qmul[cc] : -INFINITY;
+        }
+        if constexpr (MODE == kScores) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int hd = 2 * g + cc;
+            if (hd < Gu) {
+              float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap;
+              if (okR) srow[t0 + R] = sR[cc];
+              if (okR8) srow[t0 + R + 8] = sR8[cc];
+            }
+          }
+        }
+        // D4: online softmax (lazy rescale)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float tmax = fmaxf(sR[cc], sR8[cc]);
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+          if (tmax > m_run[cc] + kTau) {
+            const float alpha = ex2(m_run[cc] - tmax);
+            l_run[cc] *= alpha;
+            if constexpr (MODE == kFused) {
+#pragma unroll
+              for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                  acc[blk][mt][cc] *= alpha;
+                  acc[blk][mt][2 + cc] *= alpha;
+                }
+            }
+            m_run[cc] = tmax;
+          }
+          pR[cc] = ex2(sR[cc] - m_run[cc]);
+          pR8[cc] = ex2(sR8[cc] - m_run[cc]);
+          l_run[cc] += pR[cc] + pR8[cc];
+        }
+      } else {
+        // pass 2 of sparse-V: normalised weights from the stored scores (D5)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int hd = 2 * g + cc;
+          float wR = 0.0f, wR8 = 0.0f;
+          if (hd < Gu) {
+            const float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap;
+            if (okR) {
+              const float d2 = __ldcs(srow + t0 + R) - lse2[cc];
+              wR = d2 >= log2_thr ? ex2(d2) : 0.0f;
+            }
+            if (okR8) {
+              const float d2 = __ldcs(srow + t0 + R + 8) - lse2[cc];
+              wR8 = d2 >= log2_thr ? ex2(d2) : 0.0f;
+            }
+          }
+          pR[cc] = wR;
+          pR8[cc] = wR8;
+        }
+      }
+      if constexpr (HASV) {
+        bool any = true;
+        if constexpr (MODE == kSparseV)
+          any = __any_sync(0xffffffffu, (pR[0] + pR[1] + pR8[0] + pR8[1]) > 0.0f);
+        if (any) {
+          // D6: V accumulated in the rotated domain
+#pragma unroll
+          for (int blk = 0; blk < NB; ++blk) {
+            const uint32_t b0 = movtrans(pack_half2(pR[0] * tr.vn[0][blk], pR[1] * tr.vn[0][blk]));
+            const uint32_t b1 = movtrans(pack_half2(pR8[0] * tr.vn[1][blk], pR8[1] * tr.vn[1][blk]));
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+              const uint32_t x0 = lds(lutV, lut_off(tr.v[0][blk], 2 * VB * mt, 2 * VB, lane4));
+              const uint32_t x1 = lds(lutV, lut_off(tr.v[1][blk], 2 * VB * mt, 2 * VB, lane4));
+              const uint32_t x2 = lds(lutV, lut_off(tr.v[2][blk], 2 * VB * mt, 2 * VB, lane4));
+              const uint32_t x3 = lds(lutV, lut_off(tr.v[3][blk], 2 * VB * mt, 2 * VB, lane4));
+              mma16816(acc[blk][mt], prmt(x0, x1, 0x5410), prmt(x0, x1, 0x7632),
+                       prmt(x2, x3, 0x5410), prmt(x2, x3, 0x7632), b0, b1);
+            }
+          }
+        }
+      }
+    };
+
+    {
+      TileRegs<KB, VB, NB> ta, tb;
+      int k = seg_lo + warp;
+      if (k < seg_hi) load_tile<KB, VB, NB, HASK, HASV>(ta, up, k * kTile, lane);
+      for (;;) {
+        if (k >= seg_hi) break;
+        if (k + kWarps < seg_hi) load_tile<KB, VB, NB, HASK, HASV>(tb, up, (k + kWarps) * kTile, lane);
+        if (lane == 0 && k + (kPrefetchDist + 1) * kWarps < seg_hi)
+          prefetch_tile<KB, VB, NB, HASK, HASV>(up, (k + (kPrefetchDist + 1) * kWarps) * kTile, p.seq_cap);
+        compute(ta, k);
+        k += kWarps;
+        if (k >= seg_hi) break;
+        if (k + kWarps < seg_hi) load_tile<KB, VB, NB, HASK, HASV>(ta, up, (k + kWarps) * kTile, lane);
+        if (lane == 0 && k + (kPrefetchDist + 1) * kWarps < seg_hi)
+          prefetch_tile<KB, VB, NB, HASK, HASV>(up, (k + (kPrefetchDist + 1) * kWarps) * kTile, p.seq_cap);
+        compute(tb, k);
+        k += kWarps;
+      }
+    }
+
+    // ---- warp partials to shared memory -----------------------------------
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      float l = l_run[cc];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      if (R == 0) {
+        w_m[warp * kMaxGroup + 2 * g + cc] = m_run[cc];
+        w_l[warp * kMaxGroup + 2 * g + cc] = l;
+      }
+    }
+    if constexpr (HASV) {
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int d0 = blk * kBlock + 16 * R + 2 * mt;
+          float* w0 = work + (warp * kMaxGroup + 2 * g) * D + d0;
+          float* w1 = work + (warp * kMaxGroup + 2 * g + 1) * D + d0;
+          *reinterpret_cast<float2*>(w0) = make_float2(acc[blk][mt][0], acc[blk][mt][2]);
+          *reinterpret_cast<float2*>(w1) = make_float2(acc[blk][mt][1], acc[blk][mt][3]);
+        }
+    }
+    __syncthreads();
+
+    // ---- merge the warps in a fixed order ----------------------------------
+    if constexpr (HASK) {
+      if (tid < Gu) {
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, w_m[w * kMaxGroup + tid]);
+        float L = 0.0f;
+        for (int w = 0; w < kWarps; ++w) {
+          const float mw = w_m[w * kMaxGroup + tid];
+          if (mw != -INFINITY) L += w_l[w * kMaxGroup + tid] * ex2(mw - M);
+        }
+        u_M[tid] = M;
+        u_L[tid] = L;
+      }
+    }
+    if constexpr (HASV) {
+      for (int i = tid; i < Gu * D; i += kThreads) {
+        const int hd = i / D, d = i % D;
+        float M = 0.0f;
+        if constexpr (HASK) {
+          M = -INFINITY;
+          for (int w = 0; w < kWarps; ++w) M = fmaxf(M, w_m[w * kMaxGroup + hd]);
+        }
+        float s = 0.0f;
+        for (int w = 0; w < kWarps; ++w) {
+          float f = 1.0f;
+          if constexpr (HASK) {
+            const float mw = w_m[w * kMaxGroup + hd];
+            f = (mw == -INFINITY) ? 0.0f : ex2(mw - M);
+          }
+          s = fmaf(work[(w * kMaxGroup + hd) * D + d], f, s);
+        }
+        res[i] = s;
+      }
+    }
+    __syncthreads();
+
+    const bool whole = (seg_lo == 0 && seg_hi == nt);
+    bool finalize = false;
+    if (whole && MODE != kScores) {
+      finalize = true;  // this CTA saw the entire unit: no partial needed
+    } else {
+      // ---- publish the partial, count tiles, the last CTA merges ----------
+      const long long slot = blockIdx.x + unit;
+      if constexpr (HASK) {
+        if (tid < Gu) {
+          p.slot_ml[(slot * kMaxGroup + tid) * 2] = u_M[tid];
+          p.slot_ml[(slot * kMaxGroup + tid) * 2 + 1] = u_L[tid];
+        }
+      }
+      if constexpr (HASV) {
+        for (int i = tid; i < Gu * D; i += kThreads)
+          p.slot_acc[(slot * kMaxGroup + i / D) * D + i % D] = res[i];
+      }
+      if constexpr (MODE != kScores) {
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+          const unsigned add = (unsigned)(seg_hi - seg_lo);
+          const unsigned old = atomicAdd(p.tickets + unit, add);
+          flag[0] = (old + add == (unsigned)nt) ? 1 : 0;
+        }
+        __syncthreads();
+        finalize = flag[0] != 0;
+        if (finalize) {
+          __threadfence();
+          const long long c_first = cta_of(Su, P), c_last = cta_of(Su + nt - 1, P);
+          if constexpr (HASK) {
+            if (tid < Gu) {
+              float M = -INFINITY;
+              for (long long c = c_first; c <= c_last; ++c) {
+                if (c * T / P == (c + 1) * T / P) continue;
+                M = fmaxf(M, __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2));
+              }
+              float L = 0.0f;
+              for (long long c = c_first; c <= c_last; ++c) {
+                if (c * T / P == (c + 1) * T / P) continue;
+                const float* ml = p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2;
+                const float mc = __ldcg(ml);
+                if (mc != -INFINITY) L += __ldcg(ml + 1) * ex2(mc - M);
+              }
+              u_M[tid] = M;
+              u_L[tid] = L;
+            }
+            __syncthreads();
+          }
+          for (int i = tid; i < Gu * D; i += kThreads) {
+            const int hd = i / D, d = i % D;
+            float s = 0.0f;
+            for (long long c = c_first; c <= c_last; ++c) {
+              if (c * T / P == (c + 1) * T / P) continue;
+              float f = 1.0f;
+              if constexpr (HASK) {
+                const float mc = __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + hd) * 2);
+                f = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[hd]);
+              }
+              s = fmaf(__ldcg(p.slot_acc + ((c + unit) * kMaxGroup + hd) * D + d), f, s);
+            }
+            res[i] = s;
+          }
+          if (tid == 0) p.tickets[unit] = 0u;
+          __syncthreads();
+        }
+      }
+    }
+
+    if (finalize) {
+      // ---- D7/D8: one inverse rotation per head, o = s o (H.acc) / L -----
+      for (int s = 1; s < kBlock; s <<= 1) {
+        for (int i = tid; i < Gu * D / 2; i += kThreads) {
+          const int hd = i / (D / 2), rem = i % (D / 2);
+          const int a = (rem / s) * 2 * s + (rem % s);
+          float* row = res + hd * D;
+          const float u = row[a], w = row[a + s];
+          row[a] = u + w;
+          row[a + s] = u - w;
+        }
+        __syncthreads();
+      }
+      for (int i = tid; i < Gu * D; i += kThreads) {
+        const int hd = i / D, d = i % D;
+        const int e = d & (kBlock - 1);
+        float v = res[i];
+        if constexpr (MODE == kFused) v = v / u_L[hd];
+        if ((p.sign_mask[e >> 5] >> (e & 31)) & 1u) v = -v;
+        p.out[((size_t)b * p.q_heads + h0 + hd) * D + d] = v;
+      }
+    }
+    __syncthreads();
+    x = Su + seg_hi;
+  }
+}
+
+// --------------------------------------------------------------- launching --
+
+template <int KB, int VB, int NB, int MODE>
+int run(const DecodeParams& p, cudaStream_t stream, int p1_ctas, int* ctas_out) {
+  using SM = Smem<KB, VB, NB, MODE>;
+  const size_t smem = SM::bytes(p.batch);
+  auto kern = decode_kernel<KB, VB, NB, MODE>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+  static int cached_sms[64] = {0};
+  static int cached_occ[64] = {0};
+  static size_t cached_smem[64] = {0};
+  if (dev >= 64) return TQ_ERR_UNSUPPORTED;
+  if (cached_sms[dev] == 0 || cached_smem[dev] != smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    int sms = 0, occ = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    if (occ < 1) return TQ_ERR_UNSUPPORTED;
+    cached_occ[dev] = occ;
+    cached_smem[dev] = smem;
+    cached_sms[dev] = sms;
+  }
+  const int ctas = min(kMaxCtas, cached_sms[dev] * cached_occ[dev]);
+  kern<<<ctas, kThreads, smem, stream>>>(p, p1_ctas);
+  if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
+  if (ctas_out) *ctas_out = ctas;
+  return TQ_OK;
+}
+
+template <int KB, int VB, int NB>
+int dispatch_modes(const DecodeParams& p, cudaStream_t stream) {
+  if (p.sparse_thr > 0.0f) {
+    int p1 = 0;
+    int st = run<KB, 2, NB, kScores>(p, stream, 0, &p1);
+    if (st != TQ_OK) return st;
+    return run<2, VB, NB, kSparseV>(p, stream, p1, nullptr);
+  }
+  return run<KB, VB, NB, kFused>(p, stream, 0, nullptr);
+}
+
+template <int KB, int VB>
+int dispatch_nb(const DecodeParams& p, cudaStream_t stream) {
+  switch (p.head_dim / kBlock) {
+    case 1: return dispatch_modes<KB, VB, 1>(p, stream);
+    case 2: return dispatch_modes<KB, VB, 2>(p, stream);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+template <int KB>
+int dispatch_vb(const DecodeParams& p, cudaStream_t stream) {
+  switch (p.v_bits) {
+    case 2: return dispatch_nb<KB, 2>(p, stream);
+    case 3: return dispatch_nb<KB, 3>(p, stream);
+    case 4: return dispatch_nb<KB, 4>(p, stream);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int launch_decode(const DecodeParams& p, cudaStream_t stream) {
+  switch (p.k_bits) {
+    case 2: return dispatch_vb<2>(p, stream);
+    case 3: return dispatch_vb<3>(p, stream);
+    case 4: return dispatch_vb<4>(p, stream);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace tq

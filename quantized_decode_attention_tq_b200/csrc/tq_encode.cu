@@ -1,0 +1,241 @@
+// Encoder kernel: sign flip, fast Walsh-Hadamard transform, fp16 block norm,
+// Lloyd-Max quantisation and bit packing of 128-element KV blocks.
+//
+// Method: "TheTom/llama-cpp-turboquant" README, table "量化类型" (WHT rotation
+// then codebook quantisation on 128-element blocks); intelliparadigm
+// TurboQuant article §3.2 (H_random from a random +-1 diagonal and the
+// Hadamard matrix, fast transform in O(d log d)) and §3.3 (Lloyd-Max).
+//
+// Mapping: two lanes per 128-block, lane h holding elements [64h, 64h+64)
+// as 32 float2 registers.  Six butterfly stages run in registers (five of
+// them on packed f32x2 arithmetic), the seventh pairs the two lanes through
+// one shuffle per element.  A lane's 64 codes are contiguous in the packed
+// bitstream (8*b bytes at byte 8*b*h), so stores are plain vector stores.
+
+#include <cuda_fp16.h>
+
+#include "../../include/tq.h"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int kEncThreads = 256;
+
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+// Apply the sign of element i: bit i of the 64-bit mask set means s_i = -1.
+__device__ __forceinline__ float apply_sign(float x, uint32_t word, int bit) {
+  return __uint_as_float(__float_as_uint(x) ^ ((word << (31 - bit)) & 0x80000000u));
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t (&w)[2 * BITS]) {
+  if constexpr (BITS == 4) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else if constexpr (BITS == 3) {
+    uint2* d = reinterpret_cast<uint2*>(dst);
+    d[0] = make_uint2(w[0], w[1]);
+    d[1] = make_uint2(w[2], w[3]);
+    d[2] = make_uint2(w[4], w[5]);
+  } else {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <int BITS, bool F16, int SIDE>
+__device__ __forceinline__ void encode_side(const EncodeParams& p) {
+  constexpr int L = 1 << BITS;
+  constexpr int NPOS = L / 2 - 1;  // positive decision boundaries
+  const void* in = p.in[SIDE];
+  const int lane = threadIdx.x & 31;
+  const int h = lane & 1;
+  const int nb = p.head_dim / kBlock;
+  const long long n_blocks = (long long)p.batch * p.kv_heads * p.seq_new * nb;
+  const long long blk = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 1;
+  const bool valid = blk < n_blocks;
+
+  int b = 0, j = 0, t = 0;
+  long long row = 0, bh = 0;
+  if (valid) {
+    j = (int)(blk % nb);
+    row = blk / nb;
+    t = (int)(row % p.seq_new);
+    bh = row / p.seq_new;
+    b = (int)(bh / p.kv_heads);
+  }
+  int pos = t;
+  if (valid && p.start_pos) pos += __ldg(p.start_pos + b);
+  const bool ok = valid && pos >= 0 && pos < p.seq_cap;
+  if (valid && !ok && h == 0 && p.status) atomicOr(p.status, TQ_DEV_POS_RANGE);
+
+  // ---- load 64 elements (E1), convert to fp32 --------------------------
+  float2 x[32];
+  if constexpr (F16) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(in) +
+                                                      (row * p.head_dim + j * kBlock + 64 * h));
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint4 v = ok ? __ldcs(src + c) : make_uint4(0, 0, 0, 0);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __half2 hv = *reinterpret_cast<const __half2*>(&wv[e]);
+        x[c * 4 + e] = __half22float2(hv);
+      }
+    }
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(in) +
+                                                        (row * p.head_dim + j * kBlock + 64 * h));
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      float4 v = ok ? __ldcs(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[2 * c] = make_float2(v.x, v.y);
+      x[2 * c + 1] = make_float2(v.z, v.w);
+    }
+  }
+
+  // ---- norm (E3): 8 partial sums then a tree, then across the lane pair --
+  float2 acc[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) acc[a] = __fmul2_rn(x[a], x[a]);
+#pragma unroll
+  for (int m = 4; m < 32; ++m) acc[m & 3] = __ffma2_rn(x[m], x[m], acc[m & 3]);
+  float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+  float2 s = __fadd2_rn(s01, s23);
+  float ss = s.x + s.y;
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  const float n = __fsqrt_rn(ss);
+
+  // ---- sign flip (E1): s o x ---------------------------------------------
+  {
+    const uint32_t w0 = h ? p.sign_mask[2] : p.sign_mask[0];
+    const uint32_t w1 = h ? p.sign_mask[3] : p.sign_mask[1];
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      const uint32_t w = (m < 16) ? w0 : w1;
+      const int bit = (2 * m) & 31;
+      x[m].x = apply_sign(x[m].x, w, bit);
+      x[m].y = apply_sign(x[m].y, w, bit + 1);
+    }
+  }
+
+  // ---- fast WHT (E2): 7 unnormalised butterfly stages ---------------------
+#pragma unroll
+  for (int m = 0; m < 32; ++m) x[m] = make_float2(x[m].x + x[m].y, x[m].x - x[m].y);
+#pragma unroll
+  for (int sp = 1; sp < 32; sp <<= 1) {  // element strides 2..32 = float2 strides 1..16
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      if ((m & sp) == 0) {
+        const float2 a = x[m], c = x[m + sp];
+        x[m] = __fadd2_rn(a, c);
+        x[m + sp] = sub2(a, c);
+      }
+    }
+  }
+  {  // stride 64: the partner lane holds the other half of the block.
+    const float sg = h ? -1.0f : 1.0f;
+    const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+      float2 o;
+      o.x = __shfl_xor_sync(0xffffffffu, x[m].x, 1);
+      o.y = __shfl_xor_sync(0xffffffffu, x[m].y, 1);
+      x[m] = __ffma2_rn(sg2, x[m], o);  // h=0: x + o ; h=1: o - x
+    }
+  }
+
+  // ---- quantise (E4): idx = #{boundaries < y / n} -------------------------
+  // With symmetric boundaries {-T_k} U {0} U {T_k}, for y > 0 the count is
+  // L/2 + #{T_k < |y|/n}; for y <= 0 it is L/2 - 1 - #{T_k < |y|/n} (an exact
+  // tie at a negative boundary is the only case where this differs from the
+  // strict count, by one, and only on the boundary itself).  Comparing |y|
+  // against T_k * n avoids a division.
+  float thr[NPOS > 0 ? NPOS : 1];
+#pragma unroll
+  for (int k = 0; k < NPOS; ++k) thr[k] = p.pos_bounds[SIDE][k] * n;
+
+  uint32_t w[2 * BITS];
+#pragma unroll
+  for (int k = 0; k < 2 * BITS; ++k) w[k] = 0;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float y = (i & 1) ? x[i >> 1].y : x[i >> 1].x;
+    const float a = fabsf(y);
+    int m = 0;
+#pragma unroll
+    for (int k = 0; k < NPOS; ++k) m += (a > thr[k]) ? 1 : 0;
+    const int lowside = L / 2 - 1 - m;
+    const uint32_t idx = (uint32_t)(y > 0.0f ? (lowside ^ (L - 1)) : lowside);
+    // ---- pack (E5): LSB-first bitstream --------------------------------
+    const int bit = BITS * i;
+    const int wi = bit >> 5, sh = bit & 31;
+    w[wi] |= idx << sh;
+    if (sh + BITS > 32) w[wi + 1] |= idx >> (32 - sh);
+  }
+
+  if (ok) {
+    const long long cache_blk = ((bh * p.seq_cap) + pos) * nb + j;
+    store_codes<BITS>(p.codes[SIDE] + cache_blk * (16 * BITS) + 8 * BITS * h, w);
+    if (h == 0) {
+      __half nh = __float2half_rn(n);
+      if (__hisinf(nh)) {
+        nh = __ushort_as_half((unsigned short)0x7BFF);
+        if (p.status) atomicOr(p.status, TQ_DEV_NORM_OVERFLOW);
+      }
+      p.norms[SIDE][cache_blk] = __half_as_ushort(nh);
+    }
+  }
+}
+
+template <int KB, int VB, bool F16>
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_constant__ EncodeParams p) {
+  if (blockIdx.y == 0) {
+    if (p.in[0]) encode_side<KB, F16, 0>(p);
+  } else {
+    if (p.in[1]) encode_side<VB, F16, 1>(p);
+  }
+}
+
+template <int KB, int VB>
+int launch_kb_vb(const EncodeParams& p, cudaStream_t stream) {
+  const long long n_blocks = (long long)p.batch * p.kv_heads * p.seq_new * (p.head_dim / kBlock);
+  const long long threads = n_blocks * 2;
+  const long long grid_x = (threads + kEncThreads - 1) / kEncThreads;
+  if (grid_x > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)grid_x, 2);
+  if (p.f16)
+    encode_kernel<KB, VB, true><<<grid, kEncThreads, 0, stream>>>(p);
+  else
+    encode_kernel<KB, VB, false><<<grid, kEncThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}
+
+template <int KB>
+int launch_kb(const EncodeParams& p, cudaStream_t stream) {
+  // A side that is not encoded keeps a valid bit width from the descriptor.
+  switch (p.bits[1]) {
+    case 2: return launch_kb_vb<KB, 2>(p, stream);
+    case 3: return launch_kb_vb<KB, 3>(p, stream);
+    case 4: return launch_kb_vb<KB, 4>(p, stream);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int launch_encode(const EncodeParams& p, cudaStream_t stream) {
+  switch (p.bits[0]) {
+    case 2: return launch_kb<2>(p, stream);
+    case 3: return launch_kb<3>(p, stream);
+    case 4: return launch_kb<4>(p, stream);
+  }
+  return TQ_ERR_UNSUPPORTED;
+}
+
+}  // namespace tq

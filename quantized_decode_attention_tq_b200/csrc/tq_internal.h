@@ -1,0 +1,68 @@
+// Internal interface between the C-ABI host layer (tq_host.cpp) and the
+// sm_100a kernels (tq_encode.cu, tq_decode.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace tq {
+
+constexpr int kBlock = 128;        // elements per rotated/quantised block
+constexpr int kTile = 16;          // tokens per decode MMA tile
+constexpr int kMaxGroup = 8;       // q-heads handled together per kv-head (MMA N = 8)
+constexpr int kMaxCtas = 1024;     // upper bound on persistent decode CTAs
+constexpr int kMaxBatch = 4096;    // decode batch limit (block-wide prefix scan)
+constexpr int kMaxHeadDim = 512;   // encoder: up to 4 blocks per vector
+constexpr int kMaxDecodeHeadDim = 256;  // decode kernels are built for 1 or 2 blocks
+
+// Encoder launch parameters (one launch writes K and V).
+struct EncodeParams {
+  const void* in[2];          // K, V inputs [B, Hkv, seq_new, D] (either may be null)
+  uint8_t* codes[2];
+  uint16_t* norms[2];
+  int bits[2];
+  float pos_bounds[2][7];     // positive decision boundaries, ascending
+  const int32_t* start_pos;   // device [B] or null
+  uint32_t* status;           // device status word or null
+  uint32_t sign_mask[4];      // bit i set <=> s_i = -1
+  int f16;                    // input dtype: 1 = fp16, 0 = fp32
+  int batch, kv_heads, head_dim, seq_cap, seq_new;
+};
+
+int launch_encode(const EncodeParams& p, cudaStream_t stream);
+
+// Decode launch parameters.
+struct DecodeParams {
+  const void* q;
+  int q_f16;
+  const uint8_t* k_codes;
+  const uint16_t* k_norms;
+  const uint8_t* v_codes;
+  const uint16_t* v_norms;
+  const int32_t* seq_lens;
+  float* out;
+  uint32_t* status;
+  // workspace views
+  uint32_t* tickets;   // [units]
+  float* slot_ml;      // [(kMaxCtas + units) * kMaxGroup * 2]
+  float* slot_acc;     // [(kMaxCtas + units) * kMaxGroup * head_dim]
+  float* scores;       // sparse only: [B, Hq, seq_cap] (log2-domain scores)
+  float kcent[16], vcent[16];
+  uint32_t sign_mask[4];
+  int k_bits, v_bits;
+  int batch, kv_heads, q_heads, head_dim, seq_cap;
+  float score_mult;    // scale * log2(e) / 128
+  float sparse_thr;    // > 0: two-pass exact sparse-V
+};
+
+// Workspace layout shared by the size query and the launcher.
+struct DecodeWorkspace {
+  size_t tickets_off, ml_off, acc_off, scores_off, total;
+};
+DecodeWorkspace decode_workspace_layout(int batch, int kv_heads, int q_heads, int head_dim,
+                                        int seq_cap, bool sparse);
+
+int launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+}  // namespace tq

@@ -1,0 +1,155 @@
+"""C-ABI host tests (CPU only): the library loads, exports every symbol that
+include/tq.h declares, its host-side codebook and sign vector agree with the
+oracle, and invalid arguments are rejected before anything is launched."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import quantized_decode_attention_tq_b200 as tq
+from quantized_decode_attention_tq_b200 import _lib
+from oracle import tq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "tq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _header_functions()
+    assert len(names) == 6
+    lib = tq.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_struct_layouts():
+    assert ctypes.sizeof(_lib.Codebook) == 4 + 16 * 4 + 15 * 4
+    assert ctypes.sizeof(_lib.KVDesc) == 32
+    assert _lib.KVDesc.sign_seed.offset == 16
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_codebook_matches_oracle(bits):
+    cb = tq.make_codebook(bits)
+    c, t = tq.codebook_arrays(cb)
+    oc, ot = O.codebook_f32(bits)
+    assert np.array_equal(c, oc)
+    # The oracle's middle boundary carries an fp64 rounding residue (~1e-16);
+    # the library's is exactly 0 by symmetry.
+    np.testing.assert_allclose(t, ot, rtol=0, atol=1e-15)
+    assert t[len(t) // 2] == 0.0
+    assert np.array_equal(c, -c[::-1]) and np.array_equal(t, -t[::-1])
+
+
+@pytest.mark.parametrize("seed", [0, 1, 1234567, 2**64 - 1])
+def test_sign_vector_matches_oracle(seed):
+    assert np.array_equal(tq.sign_vector(seed), O.sign_vector(seed).astype(np.int8))
+
+
+def test_codebook_errors():
+    lib = tq.lib()
+    assert lib.tq_make_codebook(3, None) == _lib.TQ_ERR_INVALID_ARG
+    cb = _lib.Codebook()
+    assert lib.tq_make_codebook(5, ctypes.byref(cb)) == _lib.TQ_ERR_UNSUPPORTED
+    assert lib.tq_make_codebook(0, ctypes.byref(cb)) == _lib.TQ_ERR_UNSUPPORTED
+    assert lib.tq_sign_vector(0, None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_status_string(3).decode().startswith("workspace")
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+GOOD = 0x7f0000000000  # aligned fake device addresses: never dereferenced on error paths
+
+
+def test_encode_rejects_bad_arguments_without_launch():
+    lib = tq.lib()
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+
+    def call(desc, k=GOOD, v=GOOD, dtype=1, seq_new=4, kcb=cb3, vcb=cb2, kc=GOOD, vn=GOOD, sp=None):
+        return lib.tq_encode_kv(ctypes.byref(desc) if desc is not None else None,
+                                ctypes.byref(kcb), ctypes.byref(vcb),
+                                _fake(k) if k else None, _fake(v) if v else None, dtype, seq_new,
+                                _fake(sp) if sp else None, _fake(kc) if kc else None, _fake(GOOD),
+                                _fake(GOOD), _fake(vn) if vn else None, None, None)
+
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    assert call(None) == _lib.TQ_ERR_INVALID_ARG
+    assert call(tq.kv_desc(2, 2, 96, 64, 3, 2)) == _lib.TQ_ERR_UNSUPPORTED
+    assert call(tq.kv_desc(2, 2, 128, 64, 5, 2)) == _lib.TQ_ERR_UNSUPPORTED
+    assert call(tq.kv_desc(0, 2, 128, 64, 3, 2)) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, dtype=7) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, seq_new=-1) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, k=0, v=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, kc=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, vn=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, k=GOOD + 8) == _lib.TQ_ERR_INVALID_ARG          # misaligned input
+    assert call(d, kc=GOOD + 4) == _lib.TQ_ERR_INVALID_ARG         # misaligned codes
+    assert call(d, kcb=cb2) == _lib.TQ_ERR_INVALID_ARG             # codebook bits mismatch
+    assert call(d, sp=GOOD + 2) == _lib.TQ_ERR_INVALID_ARG
+    bad = tq.make_codebook(3)
+    bad.boundaries[0] = bad.boundaries[1] + 1.0                    # not ascending
+    assert call(d, kcb=bad) == _lib.TQ_ERR_INVALID_ARG
+    assert call(d, seq_new=0) == _lib.TQ_OK                        # no-op, nothing launched
+
+
+def test_decode_rejects_bad_arguments_without_launch():
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+    need = tq.decode_workspace_size(d, 8)
+
+    def call(desc=d, hq=8, q=GOOD, qd=1, kc=GOOD, lens=GOOD, scale=0.1, thr=0.0, out=GOOD, ws=GOOD,
+             wsb=None, kcb=cb3, vcb=cb2):
+        return lib.tq_decode_attention(ctypes.byref(desc), ctypes.byref(kcb), ctypes.byref(vcb), hq,
+                                       _fake(q) if q else None, qd, _fake(kc) if kc else None,
+                                       _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                       _fake(lens) if lens else None, scale, thr,
+                                       _fake(out) if out else None, _fake(ws) if ws else None,
+                                       need if wsb is None else wsb, None, None)
+
+    assert call(hq=7) == _lib.TQ_ERR_INVALID_ARG
+    assert call(hq=1) == _lib.TQ_ERR_INVALID_ARG
+    assert call(q=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(qd=3) == _lib.TQ_ERR_INVALID_ARG
+    assert call(kc=GOOD + 1) == _lib.TQ_ERR_INVALID_ARG
+    assert call(lens=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(out=GOOD + 4) == _lib.TQ_ERR_INVALID_ARG
+    assert call(scale=math.inf) == _lib.TQ_ERR_INVALID_ARG
+    assert call(thr=math.nan) == _lib.TQ_ERR_INVALID_ARG
+    assert call(kcb=cb2) == _lib.TQ_ERR_INVALID_ARG
+    assert call(ws=0) == _lib.TQ_ERR_WORKSPACE
+    assert call(ws=GOOD + 16) == _lib.TQ_ERR_WORKSPACE
+    assert call(wsb=need - 1) == _lib.TQ_ERR_WORKSPACE
+    # sparse mode needs the score buffer: the dense size is too small
+    assert call(thr=1e-5) == _lib.TQ_ERR_WORKSPACE
+    assert call(desc=tq.kv_desc(2, 2, 384, 64, 3, 2)) in (_lib.TQ_ERR_UNSUPPORTED, _lib.TQ_ERR_WORKSPACE)
+
+
+def test_workspace_size_formula():
+    d = tq.kv_desc(8, 8, 128, 32768, 3, 3)
+    dense = tq.decode_workspace_size(d, 32)
+    sparse = tq.decode_workspace_size(d, 32, 1e-6)
+    assert dense > 0 and sparse - dense >= 8 * 32 * 32768 * 4
+    assert tq.decode_workspace_size(d, 33) == 0
+    assert tq.decode_workspace_size(tq.kv_desc(8, 8, 100, 32768, 3, 3), 32) == 0
+
+
+def test_cache_shapes_give_b_plus_one_eighth_bits():
+    for b in (2, 3, 4):
+        d = tq.kv_desc(2, 3, 256, 10, b, b)
+        s = tq.cache_shapes(d)
+        code_bytes = int(np.prod(s["k_codes"]))
+        norm_bytes = 2 * int(np.prod(s["k_norms"]))
+        values = 2 * 3 * 10 * 256
+        assert (code_bytes + norm_bytes) * 8 / values == b + 16 / 128
