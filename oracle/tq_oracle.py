@@ -296,6 +296,22 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_lens, scale: floa
     return out
 
 
+def attention_weights(q: np.ndarray, k: np.ndarray, seq_lens, scale: float):
+    """Normalised softmax weights w_t = exp(s_t - LSE), s_t = scale . q.k_t, in
+    fp64, as a dict {(b, h): w[seq_lens[b]]} (same GQA mapping as attention)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    group = q.shape[1] // k.shape[1]
+    out = {}
+    for b in range(q.shape[0]):
+        n = int(seq_lens[b])
+        for h in range(q.shape[1]):
+            s = scale * (k[b, h // group, :n] @ q[b, h])
+            w = np.exp(s - s.max()) if n else s
+            out[(b, h)] = w / w.sum() if n else w
+    return out
+
+
 def decode_dequant(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale,
                    k_bits, v_bits, k_centroids, v_centroids, signs, sparse_thr=0.0):
     """Formulation A: dequantise the whole cache, then plain attention."""

@@ -301,3 +301,15 @@ def test_sparse_skip_fraction_matches_gaussian_prediction():
     pred = np.mean(stats.norm.cdf((np.log(thr * n) + sig ** 2 / 2) / sig))
     assert abs(got - pred) < 0.004, (got, pred)
     assert 0.04 < got < 0.09
+
+
+def test_attention_weights_match_torch_softmax():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((2, 4, 128))
+    k = rng.standard_normal((2, 2, 20, 128))
+    ws = O.attention_weights(q, k, [20, 7], 0.1)
+    for (b, h), w in ws.items():
+        n = [20, 7][b]
+        ref = torch.softmax(torch.tensor(k[b, h // 2, :n] @ q[b, h]) * 0.1, dim=0).numpy()
+        np.testing.assert_allclose(w, ref, rtol=1e-12, atol=1e-15)
