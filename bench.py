@@ -278,6 +278,7 @@ def run_tq(args):
     cache0 = tq.alloc_cache(desc, dev)
     tq.encode_kv(cache0, kcb, vcb, torch.from_numpy(w.k).to(dev), torch.from_numpy(w.v).to(dev))
     torch.cuda.synchronize()
+    torch.cuda.empty_cache()  # the fp16 K/V staging copies are not needed on the device
     kvb = kv_bytes(w)
     cache_bytes = sum(t.numel() * t.element_size() for t in
                       (cache0.k_codes, cache0.k_norms, cache0.v_codes, cache0.v_norms))
