@@ -5,7 +5,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
+# TQ_LIBRARY may point at another build of the same C ABI (e.g. a tuning variant).
+LIB_PATH = os.environ.get("TQ_LIBRARY") or os.path.join(_HERE, "libtq_b200.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA = range(5)
 TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE = 1, 2, 4
