@@ -37,10 +37,21 @@
 namespace tq {
 namespace {
 
-constexpr int kWarps = 4;
+#ifndef TQ_DECODE_WARPS
+#define TQ_DECODE_WARPS 4
+#endif
+#ifndef TQ_DECODE_MIN_CTAS
+#define TQ_DECODE_MIN_CTAS 3
+#endif
+#ifndef TQ_PREFETCH_STEPS
+#define TQ_PREFETCH_STEPS 4
+#endif
+constexpr int kWarps = TQ_DECODE_WARPS;
 constexpr int kThreads = 32 * kWarps;
-constexpr float kTau = 6.0f;        // lazy-rescale threshold (log2 units)
-constexpr int kPrefetchDist = 2;    // L2 bulk prefetch, in warp-loop steps
+constexpr float kTau = 6.0f;                    // lazy-rescale threshold (log2 units)
+constexpr int kPrefetchSteps = TQ_PREFETCH_STEPS;  // L2 prefetch lead, in CTA tile groups
+constexpr int kStaticLutLimit = 40 * 1024;      // tables up to this size are static shared
+constexpr int kMergeChunk = 64;                 // partials merged per pass of the final merge
 
 enum Mode { kFused = 0, kScores = 1, kSparseV = 2 };
 
@@ -105,18 +116,26 @@ struct Fmt {
   static constexpr int kBlockBytes = 16 * B;
 };
 
-// Registers holding one 16-token tile for one lane.
-// Lane (R = lane/4, g = lane%4):
-//   K rows: tokens R and R+8, codes of dims [32g, 32g+32) of each block;
-//   V cols: tokens 2g, 2g+1, 2g+8, 2g+9, codes of dims [16R, 16R+16);
-//   norms : tokens R and R+8.
+// Token order inside a 16-token tile.  MMA row r of the score product holds
+// token pi(r): pi(R) = 2R, pi(R + 8) = 2R + 1, so lane (R = lane/4, g = lane%4)
+// holds the adjacent tokens 2R and 2R+1 (their norms are one 32-bit word).
+// The P.V product then needs, in lane g, tokens pi(2g) = 4g, pi(2g+1) = 4g+2,
+// pi(2g+8) = 4g+1 and pi(2g+9) = 4g+3 -- four adjacent tokens.
+//
+// Per lane and tile:
+//   k[rr][blk]  : codes of dims [32g, 32g+32) of token 2R+rr (KB words);
+//   v[tt][blk]  : codes of dims [16R, 16R+16) of token vtok(tt) (2 words);
+//   kn, vn      : the fp16 norms of tokens 2R and 2R+1 (NB=1: one half2
+//                 word; NB=2: one word per token holding both blocks).
 template <int KB, int VB, int NB>
 struct TileRegs {
   uint32_t k[2][NB][KB > 0 ? KB : 1];
   uint32_t v[4][NB][2];
-  float kn[2][NB];
-  float vn[2][NB];
+  uint32_t kn[NB];
+  uint32_t vn[NB];
 };
+
+__device__ __forceinline__ int vtok(int g, int tt) { return 4 * g + ((tt & 1) << 1) + (tt >> 1); }
 
 struct UnitPtrs {
   const uint8_t* kc;
@@ -126,75 +145,152 @@ struct UnitPtrs {
   int len;
 };
 
-template <int KB, int VB, int NB, bool LOADK, bool LOADV>
-__device__ __forceinline__ void load_tile(TileRegs<KB, VB, NB>& r, const UnitPtrs& u, int t0,
-                                          int lane) {
+template <int KB, int VB, int NB>
+struct LaneOffsets {
+  uint32_t k[2];   // byte offset of this lane's K words for token 2R + rr (block 0)
+  uint32_t v[4];   // byte offset of this lane's V words for token vtok(tt) (block 0)
+  uint32_t vsh;    // VB == 3: extra right shift (bits) of the loaded V words
+  __device__ __forceinline__ LaneOffsets(int lane) {
+    const int R = lane >> 2, g = lane & 3;
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) k[rr] = (uint32_t)((2 * R + rr) * NB * Fmt<KB>::kBlockBytes + g * KB * 4);
+    const int vlane = VB == 4 ? 8 * R : (VB == 3 ? 4 * ((3 * R) >> 1) : 4 * R);
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) v[tt] = (uint32_t)(vtok(g, tt) * NB * Fmt<VB>::kBlockBytes + vlane);
+    vsh = (VB == 3 && (R & 1)) ? 16u : 0u;
+  }
+};
+
+template <int B>
+__device__ __forceinline__ void load_kwords(uint32_t (&dst)[B > 0 ? B : 1], const uint8_t* src) {
+  if constexpr (B == 4) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+    dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
+  } else if constexpr (B == 3) {
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
+    dst[0] = __ldg(s); dst[1] = __ldg(s + 1); dst[2] = __ldg(s + 2);
+  } else {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
+    dst[0] = x.x; dst[1] = x.y;
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void load_vwords(uint32_t (&dst)[2], const uint8_t* src, uint32_t vsh) {
+  if constexpr (B == 4) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
+    dst[0] = x.x; dst[1] = x.y;
+  } else if constexpr (B == 3) {
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
+    uint32_t w0 = __ldg(s), w1 = __ldg(s + 1);
+    dst[0] = __funnelshift_r(w0, w1, vsh);
+    dst[1] = w1 >> vsh;
+  } else {
+    dst[0] = __ldg(reinterpret_cast<const uint32_t*>(src));
+    dst[1] = 0u;
+  }
+}
+
+// Load one tile.  FULL: all 16 tokens are inside the sequence (no checks).
+template <int KB, int VB, int NB, bool LOADK, bool LOADV, bool FULL>
+__device__ __forceinline__ void load_tile(TileRegs<KB, VB, NB>& r, const UnitPtrs& u,
+                                          const LaneOffsets<KB, VB, NB>& lo, int t0, int lane) {
   const int R = lane >> 2, g = lane & 3;
+  const int nval = u.len - t0;  // valid tokens in this tile (>= 16 when FULL)
   if constexpr (LOADK) {
+    const uint8_t* base = u.kc + (size_t)t0 * NB * Fmt<KB>::kBlockBytes;
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
-      const int t = t0 + R + 8 * rr;
-      const bool ok = t < u.len;
+      const bool ok = FULL || (2 * R + rr < nval);
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        const uint8_t* src = u.kc + ((size_t)t * NB + blk) * Fmt<KB>::kBlockBytes + g * KB * 4;
-        if constexpr (KB == 4) {
-          uint4 x = ok ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
-          r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y; r.k[rr][blk][2] = x.z; r.k[rr][blk][3] = x.w;
-        } else if constexpr (KB == 3) {
-          const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
-          r.k[rr][blk][0] = ok ? __ldg(s) : 0u;
-          r.k[rr][blk][1] = ok ? __ldg(s + 1) : 0u;
-          r.k[rr][blk][2] = ok ? __ldg(s + 2) : 0u;
+        if (ok) {
+          load_kwords<KB>(r.k[rr][blk], base + lo.k[rr] + blk * Fmt<KB>::kBlockBytes);
         } else {
-          uint2 x = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0, 0);
-          r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y;
+#pragma unroll
+          for (int i = 0; i < (KB > 0 ? KB : 1); ++i) r.k[rr][blk][i] = 0u;
         }
-        r.kn[rr][blk] = ok ? __half2float(__ushort_as_half(__ldg(u.kn + (size_t)t * NB + blk))) : 0.0f;
       }
+    }
+    const uint16_t* nb = u.kn + (size_t)(t0 + 2 * R) * NB;
+    if constexpr (NB == 1) {
+      if (FULL) {
+        r.kn[0] = __ldg(reinterpret_cast<const uint32_t*>(nb));
+      } else {
+        const uint32_t a = (2 * R < nval) ? __ldg(nb) : 0u, b = (2 * R + 1 < nval) ? __ldg(nb + 1) : 0u;
+        r.kn[0] = a | (b << 16);
+      }
+    } else {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr)
+        r.kn[rr] = (FULL || 2 * R + rr < nval) ? __ldg(reinterpret_cast<const uint32_t*>(nb + rr * NB)) : 0u;
     }
   }
   if constexpr (LOADV) {
+    const uint8_t* base = u.vc + (size_t)t0 * NB * Fmt<VB>::kBlockBytes;
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt) {
-      const int t = t0 + 2 * g + (tt & 1) + 8 * (tt >> 1);
-      const bool ok = t < u.len;
+      const bool ok = FULL || (vtok(g, tt) < nval);
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        const uint8_t* blkp = u.vc + ((size_t)t * NB + blk) * Fmt<VB>::kBlockBytes;
-        if constexpr (VB == 4) {
-          uint2 x = ok ? __ldg(reinterpret_cast<const uint2*>(blkp + 8 * R)) : make_uint2(0, 0);
-          r.v[tt][blk][0] = x.x; r.v[tt][blk][1] = x.y;
-        } else if constexpr (VB == 3) {
-          // 6 bytes at byte 6R: covered by 32-bit words (3R)/2 and (3R)/2 + 1.
-          const uint32_t* s = reinterpret_cast<const uint32_t*>(blkp) + ((3 * R) >> 1);
-          uint32_t w0 = ok ? __ldg(s) : 0u, w1 = ok ? __ldg(s + 1) : 0u;
-          if (R & 1) { w0 = __funnelshift_r(w0, w1, 16); w1 >>= 16; }
-          r.v[tt][blk][0] = w0; r.v[tt][blk][1] = w1;
+        if (ok) {
+          load_vwords<VB>(r.v[tt][blk], base + lo.v[tt] + blk * Fmt<VB>::kBlockBytes, lo.vsh);
         } else {
-          r.v[tt][blk][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(blkp) + R) : 0u;
-          r.v[tt][blk][1] = 0u;
+          r.v[tt][blk][0] = r.v[tt][blk][1] = 0u;
         }
       }
     }
+    const uint16_t* nb = u.vn + (size_t)(t0 + 2 * R) * NB;
+    if constexpr (NB == 1) {
+      if (FULL) {
+        r.vn[0] = __ldg(reinterpret_cast<const uint32_t*>(nb));
+      } else {
+        const uint32_t a = (2 * R < nval) ? __ldg(nb) : 0u, b = (2 * R + 1 < nval) ? __ldg(nb + 1) : 0u;
+        r.vn[0] = a | (b << 16);
+      }
+    } else {
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int t = t0 + R + 8 * rr;
-      const bool ok = t < u.len;
-#pragma unroll
-      for (int blk = 0; blk < NB; ++blk)
-        r.vn[rr][blk] = ok ? __half2float(__ushort_as_half(__ldg(u.vn + (size_t)t * NB + blk))) * (1.0f / kBlock) : 0.0f;
+      for (int rr = 0; rr < 2; ++rr)
+        r.vn[rr] = (FULL || 2 * R + rr < nval) ? __ldg(reinterpret_cast<const uint32_t*>(nb + rr * NB)) : 0u;
     }
   }
 }
 
-// Issue L2 prefetches for one future tile (one lane per warp).
+template <int KB, int VB, int NB, bool LOADK, bool LOADV>
+__device__ __forceinline__ void load_tile_any(TileRegs<KB, VB, NB>& r, const UnitPtrs& u,
+                                              const LaneOffsets<KB, VB, NB>& lo, int t0, int lane) {
+  if (t0 + kTile <= u.len)
+    load_tile<KB, VB, NB, LOADK, LOADV, true>(r, u, lo, t0, lane);
+  else
+    load_tile<KB, VB, NB, LOADK, LOADV, false>(r, u, lo, t0, lane);
+}
+
+// Norms of tokens 2R (x) and 2R+1 (y) for block blk, as fp32.
+template <int NB>
+__device__ __forceinline__ float2 norm_pair(const uint32_t (&w)[NB], int blk) {
+  if constexpr (NB == 1) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w[0]));
+  } else {
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&w[0]));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&w[1]));
+    return blk == 0 ? make_float2(a.x, b.x) : make_float2(a.y, b.y);
+  }
+}
+
+// L2 prefetch of the tokens [tok_lo, tok_hi) of one unit (one thread).
 template <int KB, int VB, int NB, bool PK, bool PV>
-__device__ __forceinline__ void prefetch_tile(const UnitPtrs& u, int t0, int seq_cap) {
-  const int n = min(kTile, seq_cap - t0);
-  if (n <= 0) return;
-  if constexpr (PK) prefetch_l2(u.kc + (size_t)t0 * NB * Fmt<KB>::kBlockBytes, n * NB * Fmt<KB>::kBlockBytes);
-  if constexpr (PV) prefetch_l2(u.vc + (size_t)t0 * NB * Fmt<VB>::kBlockBytes, n * NB * Fmt<VB>::kBlockBytes);
+__device__ __forceinline__ void prefetch_range(const UnitPtrs& u, int tok_lo, int tok_hi) {
+  if (tok_hi <= tok_lo) return;
+  const int n = tok_hi - tok_lo;
+  if constexpr (PK) prefetch_l2(u.kc + (size_t)tok_lo * NB * Fmt<KB>::kBlockBytes, n * NB * Fmt<KB>::kBlockBytes);
+  if constexpr (PV) prefetch_l2(u.vc + (size_t)tok_lo * NB * Fmt<VB>::kBlockBytes, n * NB * Fmt<VB>::kBlockBytes);
+  const int nn = (n * NB * 2) & ~15;  // norm bytes, whole 16-byte units
+  if (nn > 0) {
+    const uint16_t* a = u.kn + (size_t)tok_lo * NB;
+    const uint16_t* b = u.vn + (size_t)tok_lo * NB;
+    if (PK && (reinterpret_cast<uintptr_t>(a) & 15) == 0) prefetch_l2(a, nn);
+    if (PV && (reinterpret_cast<uintptr_t>(b) & 15) == 0) prefetch_l2(b, nn);
+  }
 }
 
 // ----------------------------------------------------- shared-memory plan --
@@ -206,30 +302,81 @@ struct Smem {
   static constexpr bool kHasV = MODE != kScores;
   static constexpr int kLutK = kHasK ? Fmt<KB>::kLutBytes : 0;
   static constexpr int kLutV = kHasV ? Fmt<VB>::kLutBytes : 0;
+  // Tables that fit live in static shared memory (their base then folds into
+  // the load's immediate offset); larger ones go to dynamic shared memory.
+  static constexpr bool kStaticLut = kLutK + kLutV <= kStaticLutLimit;
+  static constexpr int kStaticBytes = kStaticLut ? kLutK + kLutV : 16;
+  static constexpr int kDynLut = kStaticLut ? 0 : kLutK + kLutV;
   static constexpr int kWorkFloats = kWarps * kMaxGroup * D;     // per-warp partials / qhat
   static constexpr int kResFloats = kMaxGroup * D;               // merged rotated-domain acc
   static constexpr int kOffLutK = 0;
   static constexpr int kOffLutV = kOffLutK + kLutK;
-  static constexpr int kOffWork = kOffLutV + kLutV;
+  static constexpr int kOffDyn = kDynLut;
+  static constexpr int kOffWork = kOffDyn;
   static constexpr int kOffRes = kOffWork + kWorkFloats * 4;
   static constexpr int kOffMisc = kOffRes + kResFloats * 4;
   // misc: warp m/l [kWarps][8] x2, merged M/L/lse [8] x3, qexp [8], flag, then batch prefix.
-  static constexpr int kMiscFloats = 2 * kWarps * kMaxGroup + 4 * kMaxGroup + 4;
+  static constexpr int kMiscFloats = 2 * kWarps * kMaxGroup + 4 * kMaxGroup + 4 + 2 * kThreads +
+                                     kMergeChunk * kMaxGroup;
   static constexpr int kOffPrefix = kOffMisc + kMiscFloats * 4;
   static size_t bytes(int batch) { return (size_t)kOffPrefix + (size_t)(batch + 1) * 4; }
 };
 
+// Per-head (M, L) = (max m, sum l * 2^(m - M)) over the partials of one unit,
+// using every thread: thread t takes head t % 8 and every (kThreads/8)-th
+// partial, folding them in a fixed order; the kThreads/8 running pairs of a
+// head are then combined in a fixed order.  Partials of CTAs whose range is
+// empty are skipped.
+__device__ __forceinline__ void unit_stats(const float* slot_ml, long long c_first, long long c_last,
+                                           long long parts, long long T, long long unit, int Gu,
+                                           float* red_m, float* red_l, float* outM, float* outL) {
+  constexpr int J = kThreads / kMaxGroup;
+  const int tid = threadIdx.x, hd = tid % kMaxGroup, j = tid / kMaxGroup;
+  float m = -INFINITY, l = 0.0f;
+  if (hd < Gu) {
+    for (long long c = c_first + j; c <= c_last; c += J) {
+      if (c * T / parts == (c + 1) * T / parts) continue;
+      const float* ml = slot_ml + ((c + unit) * kMaxGroup + hd) * 2;
+      const float mc = __ldcg(ml), lc = __ldcg(ml + 1);
+      if (mc == -INFINITY) continue;
+      if (mc > m) {
+        l = l * ex2(m - mc) + lc;
+        m = mc;
+      } else {
+        l += lc * ex2(mc - m);
+      }
+    }
+  }
+  red_m[tid] = m;
+  red_l[tid] = l;
+  __syncthreads();
+  if (tid < Gu) {
+    float M = -INFINITY;
+    for (int jj = 0; jj < J; ++jj) M = fmaxf(M, red_m[jj * kMaxGroup + tid]);
+    float L = 0.0f;
+    for (int jj = 0; jj < J; ++jj) {
+      const float mj = red_m[jj * kMaxGroup + tid];
+      if (mj != -INFINITY) L += red_l[jj * kMaxGroup + tid] * ex2(mj - M);
+    }
+    outM[tid] = M;
+    outL[tid] = L;
+  }
+  __syncthreads();
+}
+
 // --------------------------------------------------------------- the kernel --
 
 template <int KB, int VB, int NB, int MODE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, TQ_DECODE_MIN_CTAS)
 decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   using SM = Smem<KB, VB, NB, MODE>;
   constexpr int D = SM::D;
   constexpr bool HASK = SM::kHasK, HASV = SM::kHasV;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* lutK = smem + SM::kOffLutK;
-  uint8_t* lutV = smem + SM::kOffLutV;
+  __shared__ __align__(128) uint8_t slut[SM::kStaticBytes];
+  uint8_t* lut_base = SM::kStaticLut ? slut : smem;
+  uint8_t* lutK = lut_base + SM::kOffLutK;
+  uint8_t* lutV = lut_base + SM::kOffLutV;
   float* work = reinterpret_cast<float*>(smem + SM::kOffWork);
   float* res = reinterpret_cast<float*>(smem + SM::kOffRes);
   float* misc = reinterpret_cast<float*>(smem + SM::kOffMisc);
@@ -240,6 +387,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   float* u_lse = u_L + kMaxGroup;                     // [8]
   int* qexp = reinterpret_cast<int*>(u_lse + kMaxGroup);  // [8]
   int* flag = qexp + kMaxGroup;
+  float* red_m = reinterpret_cast<float*>(flag + 4);  // [kThreads]
+  float* red_l = red_m + kThreads;                     // [kThreads]
+  float* fac = red_l + kThreads;                       // [kMergeChunk][8]
   int* prefix = reinterpret_cast<int*>(smem + SM::kOffPrefix);  // [B+1] tiles per batch, prefix
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -405,23 +555,13 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     if constexpr (MODE == kSparseV) {
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote
-      if (tid < Gu) {
+      {
         const long long P1 = p1_ctas;
-        const long long c_first = cta_of(Su, P1), c_last = cta_of(Su + nt - 1, P1);
-        float M = -INFINITY;
-        for (long long c = c_first; c <= c_last; ++c) {
-          if (c * T / P1 == (c + 1) * T / P1) continue;  // empty range
-          M = fmaxf(M, __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2));
-        }
-        float L = 0.0f;
-        for (long long c = c_first; c <= c_last; ++c) {
-          if (c * T / P1 == (c + 1) * T / P1) continue;
-          const float* ml = p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2;
-          L += __ldcg(ml + 1) * ex2(__ldcg(ml) - M);
-        }
-        u_lse[tid] = M + __log2f(L);
+        unit_stats(p.slot_ml, cta_of(Su, P1), cta_of(Su + nt - 1, P1), P1, T, unit, Gu, red_m, red_l,
+                   u_M, u_L);
+        if (tid < Gu) u_lse[tid] = u_M[tid] + __log2f(u_L[tid]);
+        __syncthreads();
       }
-      __syncthreads();
       lse2[0] = (2 * g < Gu) ? u_lse[2 * g] : 0.0f;
       lse2[1] = (2 * g + 1 < Gu) ? u_lse[2 * g + 1] : 0.0f;
     }
@@ -438,23 +578,27 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.0f, 0.0f};
 
+    const LaneOffsets<KB, VB, NB> loff(lane);
     auto compute = [&](const TileRegs<KB, VB, NB>& tr, int tile) {
       const int t0 = tile * kTile;
-      const bool okR = t0 + R < len, okR8 = t0 + R + 8 < len;
+      // rows R and R+8 of the score tile are tokens 2R and 2R+1
+      const bool okR = t0 + 2 * R < len, okR8 = t0 + 2 * R + 1 < len;
       float pR[2], pR8[2];
       if constexpr (HASK) {
-        // D2/D3: scores in the Hadamard domain, straight from the codes
-        float c[NB][4];
+        // D2/D3: scores in the Hadamard domain, straight from the codes; two
+        // independent accumulator chains (even / odd k-steps)
+        float ca[NB][4], cb[NB][4];
 #pragma unroll
         for (int blk = 0; blk < NB; ++blk) {
-          c[blk][0] = c[blk][1] = c[blk][2] = c[blk][3] = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ca[blk][e] = cb[blk][e] = 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint32_t a0 = lds(lutK, lut_off(tr.k[0][blk], 2 * KB * (2 * j), 2 * KB, lane4));
             const uint32_t a1 = lds(lutK, lut_off(tr.k[1][blk], 2 * KB * (2 * j), 2 * KB, lane4));
             const uint32_t a2 = lds(lutK, lut_off(tr.k[0][blk], 2 * KB * (2 * j + 1), 2 * KB, lane4));
             const uint32_t a3 = lds(lutK, lut_off(tr.k[1][blk], 2 * KB * (2 * j + 1), 2 * KB, lane4));
-            mma16816(c[blk], a0, a1, a2, a3, qf[blk][j][0], qf[blk][j][1]);
+            mma16816((j & 1) ? cb[blk] : ca[blk], a0, a1, a2, a3, qf[blk][j][0], qf[blk][j][1]);
           }
         }
         float sR[2], sR8[2];
@@ -463,8 +607,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           float a = 0.0f, bb = 0.0f;
 #pragma unroll
           for (int blk = 0; blk < NB; ++blk) {
-            a = fmaf(c[blk][cc], tr.kn[0][blk], a);
-            bb = fmaf(c[blk][2 + cc], tr.kn[1][blk], bb);
+            const float2 kn = norm_pair<NB>(tr.kn, blk);
+            a = fmaf(ca[blk][cc] + cb[blk][cc], kn.x, a);
+            bb = fmaf(ca[blk][2 + cc] + cb[blk][2 + cc], kn.y, bb);
           }
           sR[cc] = okR ? a * qmul[cc] : -INFINITY;
           sR8[cc] = okR8 ? bb * qmul[cc] : -INFINITY;
@@ -474,33 +619,44 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           for (int cc = 0; cc < 2; ++cc) {
             const int hd = 2 * g + cc;
             if (hd < Gu) {
-              float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap;
-              if (okR) srow[t0 + R] = sR[cc];
-              if (okR8) srow[t0 + R + 8] = sR8[cc];
+              float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap + t0 + 2 * R;
+              if (okR8) {
+                *reinterpret_cast<float2*>(srow) = make_float2(sR[cc], sR8[cc]);
+              } else if (okR) {
+                srow[0] = sR[cc];
+              }
             }
           }
         }
-        // D4: online softmax (lazy rescale)
+        // D4: online softmax.  The per-head maximum is only reduced across the
+        // warp when some lane's scores exceed the reference by more than 2^kTau.
+        const float lm0 = fmaxf(sR[0], sR8[0]), lm1 = fmaxf(sR[1], sR8[1]);
+        const bool need = (lm0 > m_run[0] + kTau) || (lm1 > m_run[1] + kTau);
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            float tmax = cc ? lm1 : lm0;
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+            if (tmax > m_run[cc] + kTau) {
+              const float alpha = ex2(m_run[cc] - tmax);
+              l_run[cc] *= alpha;
+              if constexpr (MODE == kFused) {
+#pragma unroll
+                for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+                  for (int mt = 0; mt < 8; ++mt) {
+                    acc[blk][mt][cc] *= alpha;
+                    acc[blk][mt][2 + cc] *= alpha;
+                  }
+              }
+              m_run[cc] = tmax;
+            }
+          }
+        }
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          float tmax = fmaxf(sR[cc], sR8[cc]);
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
-          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-          if (tmax > m_run[cc] + kTau) {
-            const float alpha = ex2(m_run[cc] - tmax);
-            l_run[cc] *= alpha;
-            if constexpr (MODE == kFused) {
-#pragma unroll
-              for (int blk = 0; blk < NB; ++blk)
-#pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                  acc[blk][mt][cc] *= alpha;
-                  acc[blk][mt][2 + cc] *= alpha;
-                }
-            }
-            m_run[cc] = tmax;
-          }
           pR[cc] = ex2(sR[cc] - m_run[cc]);
           pR8[cc] = ex2(sR8[cc] - m_run[cc]);
           l_run[cc] += pR[cc] + pR8[cc];
@@ -512,15 +668,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           const int hd = 2 * g + cc;
           float wR = 0.0f, wR8 = 0.0f;
           if (hd < Gu) {
-            const float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap;
-            if (okR) {
-              const float d2 = __ldcs(srow + t0 + R) - lse2[cc];
-              wR = d2 >= log2_thr ? ex2(d2) : 0.0f;
-            }
+            const float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap + t0 + 2 * R;
+            float s0 = -INFINITY, s1 = -INFINITY;
             if (okR8) {
-              const float d2 = __ldcs(srow + t0 + R + 8) - lse2[cc];
-              wR8 = d2 >= log2_thr ? ex2(d2) : 0.0f;
+              const float2 sv = __ldcs(reinterpret_cast<const float2*>(srow));
+              s0 = sv.x;
+              s1 = sv.y;
+            } else if (okR) {
+              s0 = __ldcs(srow);
             }
+            const float d0 = s0 - lse2[cc], d1 = s1 - lse2[cc];
+            wR = d0 >= log2_thr ? ex2(d0) : 0.0f;
+            wR8 = d1 >= log2_thr ? ex2(d1) : 0.0f;
           }
           pR[cc] = wR;
           pR8[cc] = wR8;
@@ -534,8 +693,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           // D6: V accumulated in the rotated domain
 #pragma unroll
           for (int blk = 0; blk < NB; ++blk) {
-            const uint32_t b0 = movtrans(pack_half2(pR[0] * tr.vn[0][blk], pR[1] * tr.vn[0][blk]));
-            const uint32_t b1 = movtrans(pack_half2(pR8[0] * tr.vn[1][blk], pR8[1] * tr.vn[1][blk]));
+            const float2 vn = norm_pair<NB>(tr.vn, blk);
+            const float sv0 = vn.x * (1.0f / kBlock), sv1 = vn.y * (1.0f / kBlock);
+            const uint32_t b0 = movtrans(pack_half2(pR[0] * sv0, pR[1] * sv0));
+            const uint32_t b1 = movtrans(pack_half2(pR8[0] * sv1, pR8[1] * sv1));
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
               const uint32_t x0 = lds(lutV, lut_off(tr.v[0][blk], 2 * VB * mt, 2 * VB, lane4));
@@ -551,22 +712,33 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     };
 
     {
+      // Warp w takes tiles seg_lo + w, seg_lo + w + kWarps, ...; one thread
+      // keeps the L2 kPrefetchSteps tile groups ahead of the CTA.
+      const bool pf_thread = (tid == 0);
+      auto prefetch_group = [&](int first_tile) {
+        const int a = max(first_tile, seg_lo), e = min(first_tile + kWarps, seg_hi);
+        if (a < e) prefetch_range<KB, VB, NB, HASK, HASV>(up, a * kTile, min(e * kTile, len));
+      };
+      if (pf_thread)
+        prefetch_range<KB, VB, NB, HASK, HASV>(up, seg_lo * kTile,
+                                               min(min(seg_hi, seg_lo + (kPrefetchSteps + 1) * kWarps) * kTile, len));
       TileRegs<KB, VB, NB> ta, tb;
       int k = seg_lo + warp;
-      if (k < seg_hi) load_tile<KB, VB, NB, HASK, HASV>(ta, up, k * kTile, lane);
+      int step = 0;
+      if (k < seg_hi) load_tile_any<KB, VB, NB, HASK, HASV>(ta, up, loff, k * kTile, lane);
       for (;;) {
         if (k >= seg_hi) break;
-        if (k + kWarps < seg_hi) load_tile<KB, VB, NB, HASK, HASV>(tb, up, (k + kWarps) * kTile, lane);
-        if (lane == 0 && k + (kPrefetchDist + 1) * kWarps < seg_hi)
-          prefetch_tile<KB, VB, NB, HASK, HASV>(up, (k + (kPrefetchDist + 1) * kWarps) * kTile, p.seq_cap);
+        if (k + kWarps < seg_hi) load_tile_any<KB, VB, NB, HASK, HASV>(tb, up, loff, (k + kWarps) * kTile, lane);
+        if (pf_thread) prefetch_group(seg_lo + (step + kPrefetchSteps + 1) * kWarps);
         compute(ta, k);
         k += kWarps;
+        ++step;
         if (k >= seg_hi) break;
-        if (k + kWarps < seg_hi) load_tile<KB, VB, NB, HASK, HASV>(ta, up, (k + kWarps) * kTile, lane);
-        if (lane == 0 && k + (kPrefetchDist + 1) * kWarps < seg_hi)
-          prefetch_tile<KB, VB, NB, HASK, HASV>(up, (k + (kPrefetchDist + 1) * kWarps) * kTile, p.seq_cap);
+        if (k + kWarps < seg_hi) load_tile_any<KB, VB, NB, HASK, HASV>(ta, up, loff, (k + kWarps) * kTile, lane);
+        if (pf_thread) prefetch_group(seg_lo + (step + kPrefetchSteps + 1) * kWarps);
         compute(tb, k);
         k += kWarps;
+        ++step;
       }
     }
 
@@ -662,38 +834,38 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         if (finalize) {
           __threadfence();
           const long long c_first = cta_of(Su, P), c_last = cta_of(Su + nt - 1, P);
-          if constexpr (HASK) {
-            if (tid < Gu) {
-              float M = -INFINITY;
-              for (long long c = c_first; c <= c_last; ++c) {
-                if (c * T / P == (c + 1) * T / P) continue;
-                M = fmaxf(M, __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2));
+          if constexpr (HASK) unit_stats(p.slot_ml, c_first, c_last, P, T, unit, Gu, red_m, red_l, u_M, u_L);
+          for (int i = tid; i < Gu * D; i += kThreads) res[i] = 0.0f;
+          for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
+            // weights 2^(m_c - M) of this chunk's partials (0 for empty ranges)
+            for (int i = tid; i < kMergeChunk * kMaxGroup; i += kThreads) {
+              const long long c = c0 + i / kMaxGroup;
+              const int hd = i % kMaxGroup;
+              float f = 0.0f;
+              if (c <= c_last && hd < Gu && c * T / P != (c + 1) * T / P) {
+                f = 1.0f;
+                if constexpr (HASK) {
+                  const float mc = __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + hd) * 2);
+                  f = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[hd]);
+                }
               }
-              float L = 0.0f;
-              for (long long c = c_first; c <= c_last; ++c) {
-                if (c * T / P == (c + 1) * T / P) continue;
-                const float* ml = p.slot_ml + ((c + unit) * kMaxGroup + tid) * 2;
-                const float mc = __ldcg(ml);
-                if (mc != -INFINITY) L += __ldcg(ml + 1) * ex2(mc - M);
-              }
-              u_M[tid] = M;
-              u_L[tid] = L;
+              fac[i] = f;
             }
             __syncthreads();
-          }
-          for (int i = tid; i < Gu * D; i += kThreads) {
-            const int hd = i / D, d = i % D;
-            float s = 0.0f;
-            for (long long c = c_first; c <= c_last; ++c) {
-              if (c * T / P == (c + 1) * T / P) continue;
-              float f = 1.0f;
-              if constexpr (HASK) {
-                const float mc = __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + hd) * 2);
-                f = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[hd]);
+            const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
+            for (int i = tid; i < Gu * D; i += kThreads) {
+              const int hd = i / D, d = i % D;
+              const float* src = p.slot_acc + ((c0 + unit) * kMaxGroup + hd) * D + d;
+              float sacc = res[i];
+#pragma unroll 8
+              for (int cc = 0; cc < n; ++cc) {
+                const float f = fac[cc * kMaxGroup + hd];
+                const float a = __ldcg(src + (size_t)cc * kMaxGroup * D);
+                sacc = (f != 0.0f) ? fmaf(a, f, sacc) : sacc;
               }
-              s = fmaf(__ldcg(p.slot_acc + ((c + unit) * kMaxGroup + hd) * D + d), f, s);
+              res[i] = sacc;
             }
-            res[i] = s;
+            __syncthreads();
           }
           if (tid == 0) p.tickets[unit] = 0u;
           __syncthreads();
