@@ -241,9 +241,8 @@ def run_tq(args):
 
     import quantized_decode_attention_tq_b200 as tq
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from quantized_decode_attention_tq_b200 import dist as tqd
+    rank, local, world = tqd.rank_info()
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
     torch.cuda.set_device(local)
@@ -257,20 +256,12 @@ def run_tq(args):
             dist.barrier()
 
     def allmax(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return tqd.reduce_max(x, dev)
 
     def allsum(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+        return tqd.reduce_sum(x, dev)
 
-    w = workload(args.workload, rank)
+    w = workload(args.workload, tqd.workload_seed(rank))
     desc = tq.kv_desc(w.batch, w.kv_heads, w.head_dim, w.seq_cap, w.k_bits, w.v_bits, w.sign_seed)
     kcb, vcb = tq.make_codebook(w.k_bits), tq.make_codebook(w.v_bits)
 
