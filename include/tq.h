@@ -59,7 +59,8 @@ typedef enum {
   TQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment           */
   TQ_ERR_UNSUPPORTED = 2,  /* valid but not built: bits, head_dim, group     */
   TQ_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required     */
-  TQ_ERR_CUDA = 4          /* a CUDA runtime call failed (launch, attribute) */
+  TQ_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute) */
+  TQ_ERR_SCRATCH_LIMIT = 5 /* needs more than the built-in scratch array      */
 } tq_status;
 
 /* Bits of the device status word (sticky; the library only ORs into it). */
@@ -173,6 +174,39 @@ int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const t
                         const int32_t* seq_lens, float scale, float sparse_thr, float* out,
                         void* workspace, size_t workspace_bytes, uint32_t* dev_status,
                         void* stream);
+
+/*
+ * tq_decode_attention_noalloc -- tq_decode_attention for callers that must
+ * not allocate device memory.  The pages have no counterpart: this is a
+ * deployment variant of the same decode kernels, not a step of the method.
+ *
+ * Who needs it: code that receives its device buffers from a host application
+ * owning all device memory (a plugin inside a serving engine with its own
+ * pool, a component with a fixed memory budget) cannot call cudaMalloc, or
+ * cannot afford the device synchronisation an allocation may cause, and so
+ * cannot supply a workspace.  This entry point takes the same arguments as
+ * tq_decode_attention minus the workspace and allocates nothing: its scratch
+ * is a fixed array of TQ_NOALLOC_SCRATCH_BYTES (64 MiB) built into the
+ * library, which every GPU that loads the library holds until exit.
+ *   - Limit: when tq_decode_workspace_size(desc, q_heads, sparse_thr) exceeds
+ *     TQ_NOALLOC_SCRATCH_BYTES it returns TQ_ERR_SCRATCH_LIMIT and launches
+ *     nothing.  Other argument errors are those of tq_decode_attention.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (with that device current); make that first call before any
+ *     stream capture.  Later calls do no set-up.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     last call's contents; each call clears the counters that must start at
+ *     zero (one cudaMemsetAsync on `stream`, no allocation).  Calls whose
+ *     executions overlap on the GPU (different streams, or concurrent host
+ *     threads) race on the array and give wrong results: serialise them.
+ */
+#define TQ_NOALLOC_SCRATCH_BYTES (64u << 20)
+int tq_decode_attention_noalloc(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                                const tq_codebook* v_cb, int q_heads, const void* q, int q_dtype,
+                                const uint8_t* k_codes, const uint16_t* k_norms,
+                                const uint8_t* v_codes, const uint16_t* v_norms,
+                                const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                                uint32_t* dev_status, void* stream);
 
 /* Static description of a status code. */
 const char* tq_status_string(int status);

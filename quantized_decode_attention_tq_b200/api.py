@@ -136,3 +136,22 @@ def decode_attention(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, 
         _ptr(status, "status"), _stream(stream))
     check("tq_decode_attention", st)
     return out
+
+
+def decode_attention_noalloc(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, scale: float,
+                             out, sparse_thr: float = 0.0, status=None, stream=None):
+    """Decode attention without a caller workspace (tq_decode_attention_noalloc).
+
+    For callers that may not allocate device memory: the library's built-in
+    64 MiB scratch array is used instead.  Calls must not overlap on the GPU.
+    """
+    q_heads = q.shape[1]
+    st = lib().tq_decode_attention_noalloc(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb), q_heads,
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention_noalloc", st)
+    return out

@@ -279,6 +279,7 @@ const char* tq_status_string(int status) {
     case TQ_ERR_UNSUPPORTED: return "unsupported configuration";
     case TQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case TQ_ERR_CUDA: return "CUDA runtime error";
+    case TQ_ERR_SCRATCH_LIMIT: return "request needs more than the built-in no-alloc scratch array";
     default: return "unknown status";
   }
 }

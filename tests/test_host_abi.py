@@ -24,7 +24,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol():
     names = _header_functions()
-    assert len(names) == 6
+    assert len(names) == 7
     lib = tq.lib()
     for n in names:
         assert hasattr(lib, n), n
