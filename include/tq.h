@@ -153,8 +153,9 @@ size_t tq_decode_workspace_size(const tq_kv_desc* desc, int q_heads, float spars
  * Sparse-V (sparse_thr > 0): positions with w_t < sparse_thr (w the
  * normalised weight) contribute zero and the rest are not renormalised.
  *
- * Supported: head_dim 128 or 256 (TQ_ERR_UNSUPPORTED otherwise), batch <=
- * 4096, any q_heads / kv_heads ratio (groups above 8 run in slices of 8).
+ * Supported: head_dim 128 or 256, an even seq_cap, batch <= 4096
+ * (TQ_ERR_UNSUPPORTED otherwise), and any q_heads / kv_heads ratio (groups
+ * above 8 run in slices of 8).
  * q: device [batch, q_heads, head_dim], q_dtype TQ_F32 or TQ_F16.
  *    q_heads must be a multiple of kv_heads.
  * seq_lens: device int32 [batch]; values are clamped to [0, seq_cap]

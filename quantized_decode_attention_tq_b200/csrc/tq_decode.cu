@@ -14,6 +14,11 @@
 //    (m, l, acc) per unit it touches; the CTA that completes a unit (atomic
 //    tile count) merges the partials in a fixed order and applies the inverse
 //    rotation, so results do not depend on scheduling.
+//  * Each warp streams its own future tiles (packed K and V codes and their
+//    fp16 norms) into a private shared-memory ring with 16-byte cp.async
+//    (zero-filled past the end of the sequence) and waits for them with
+//    cp.async.wait_group, so several tiles per warp are in flight without
+//    holding registers, and no warp waits on another.
 //  * Scores: S[16 tok x 8 heads] = Kc[16 x 128] . Qhat[128 x 8] with
 //    mma.sync m16n8k16 (f16 in, f32 accumulate).  K codes are turned into f16
 //    A fragments in registers through a shared-memory table indexed by two
@@ -43,13 +48,14 @@ namespace {
 #ifndef TQ_DECODE_MIN_CTAS
 #define TQ_DECODE_MIN_CTAS 3
 #endif
-#ifndef TQ_PREFETCH_STEPS
-#define TQ_PREFETCH_STEPS 4
+#ifndef TQ_RING_DEPTH
+#define TQ_RING_DEPTH 4
 #endif
-constexpr int kWarps = TQ_DECODE_WARPS;
-constexpr int kThreads = 32 * kWarps;
+constexpr int kCWarps = TQ_DECODE_WARPS;        // warps per CTA
+constexpr int kCThreads = 32 * kCWarps;
+constexpr int kThreads = kCThreads;
+constexpr int kDepth = TQ_RING_DEPTH;           // tiles per warp ring (in flight: kDepth - 1)
 constexpr float kTau = 6.0f;                    // lazy-rescale threshold (log2 units)
-constexpr int kPrefetchSteps = TQ_PREFETCH_STEPS;  // L2 prefetch lead, in CTA tile groups
 constexpr int kStaticLutLimit = 40 * 1024;      // tables up to this size are static shared
 constexpr int kMergeChunk = 64;                 // partials merged per pass of the final merge
 
@@ -87,8 +93,8 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
 // Byte offset into a lane-replicated table: field of `fb` bits at bit `pos`
@@ -108,6 +114,29 @@ __device__ __forceinline__ uint32_t lut_off(const uint32_t* w, int pos, int fb, 
 __device__ __forceinline__ uint32_t lds(const uint8_t* base, uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(base + off);
 }
+
+// ---------------------------------------------------------- async copies --
+
+// 16-byte global -> shared copy; src_bytes < 16 zero-fills the rest (0: no read).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+// 4-byte global -> shared copy with the same zero-fill rule.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void consumer_sync() { __syncthreads(); }
 
 template <int B>
 struct Fmt {
@@ -135,134 +164,67 @@ struct TileRegs {
   uint32_t vn[NB];
 };
 
-__device__ __forceinline__ int vtok(int g, int tt) { return 4 * g + ((tt & 1) << 1) + (tt >> 1); }
-
-struct UnitPtrs {
-  const uint8_t* kc;
-  const uint16_t* kn;
-  const uint8_t* vc;
-  const uint16_t* vn;
-  int len;
-};
-
-template <int KB, int VB, int NB>
-struct LaneOffsets {
-  uint32_t k[2];   // byte offset of this lane's K words for token 2R + rr (block 0)
-  uint32_t v[4];   // byte offset of this lane's V words for token vtok(tt) (block 0)
-  uint32_t vsh;    // VB == 3: extra right shift (bits) of the loaded V words
-  __device__ __forceinline__ LaneOffsets(int lane) {
-    const int R = lane >> 2, g = lane & 3;
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) k[rr] = (uint32_t)((2 * R + rr) * NB * Fmt<KB>::kBlockBytes + g * KB * 4);
-    const int vlane = VB == 4 ? 8 * R : (VB == 3 ? 4 * ((3 * R) >> 1) : 4 * R);
-#pragma unroll
-    for (int tt = 0; tt < 4; ++tt) v[tt] = (uint32_t)(vtok(g, tt) * NB * Fmt<VB>::kBlockBytes + vlane);
-    vsh = (VB == 3 && (R & 1)) ? 16u : 0u;
-  }
-};
-
-template <int B>
-__device__ __forceinline__ void load_kwords(uint32_t (&dst)[B > 0 ? B : 1], const uint8_t* src) {
-  if constexpr (B == 4) {
-    const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
-    dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
-  } else if constexpr (B == 3) {
-    const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
-    dst[0] = __ldg(s); dst[1] = __ldg(s + 1); dst[2] = __ldg(s + 2);
-  } else {
-    const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
-    dst[0] = x.x; dst[1] = x.y;
-  }
-}
-
-template <int B>
-__device__ __forceinline__ void load_vwords(uint32_t (&dst)[2], const uint8_t* src, uint32_t vsh) {
-  if constexpr (B == 4) {
-    const uint2 x = __ldg(reinterpret_cast<const uint2*>(src));
-    dst[0] = x.x; dst[1] = x.y;
-  } else if constexpr (B == 3) {
-    const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
-    uint32_t w0 = __ldg(s), w1 = __ldg(s + 1);
-    dst[0] = __funnelshift_r(w0, w1, vsh);
-    dst[1] = w1 >> vsh;
-  } else {
-    dst[0] = __ldg(reinterpret_cast<const uint32_t*>(src));
-    dst[1] = 0u;
-  }
-}
-
-// Load one tile.  FULL: all 16 tokens are inside the sequence (no checks).
-template <int KB, int VB, int NB, bool LOADK, bool LOADV, bool FULL>
-__device__ __forceinline__ void load_tile(TileRegs<KB, VB, NB>& r, const UnitPtrs& u,
-                                          const LaneOffsets<KB, VB, NB>& lo, int t0, int lane) {
-  const int R = lane >> 2, g = lane & 3;
-  const int nval = u.len - t0;  // valid tokens in this tile (>= 16 when FULL)
+// Code words of one tile from a ring stage.  ks / vs point at this lane's
+// first K / V word of the warp's tile (see the lane offsets in the kernel).
+template <int KB, int VB, int NB, bool LOADK, bool LOADV>
+__device__ __forceinline__ void read_tile(TileRegs<KB, VB, NB>& r, const uint8_t* ks, const uint8_t* vs,
+                                          int R) {
   if constexpr (LOADK) {
-    const uint8_t* base = u.kc + (size_t)t0 * NB * Fmt<KB>::kBlockBytes;
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const bool ok = FULL || (2 * R + rr < nval);
+    for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        if (ok) {
-          load_kwords<KB>(r.k[rr][blk], base + lo.k[rr] + blk * Fmt<KB>::kBlockBytes);
+        const uint8_t* s = ks + (rr * NB + blk) * Fmt<KB>::kBlockBytes;
+        if constexpr (KB == 4) {
+          const uint4 x = *reinterpret_cast<const uint4*>(s);
+          r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y; r.k[rr][blk][2] = x.z; r.k[rr][blk][3] = x.w;
+        } else if constexpr (KB == 3) {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(s);
+          r.k[rr][blk][0] = w[0]; r.k[rr][blk][1] = w[1]; r.k[rr][blk][2] = w[2];
         } else {
-#pragma unroll
-          for (int i = 0; i < (KB > 0 ? KB : 1); ++i) r.k[rr][blk][i] = 0u;
+          const uint2 x = *reinterpret_cast<const uint2*>(s);
+          r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y;
         }
       }
-    }
-    const uint16_t* nb = u.kn + (size_t)(t0 + 2 * R) * NB;
-    if constexpr (NB == 1) {
-      if (FULL) {
-        r.kn[0] = __ldg(reinterpret_cast<const uint32_t*>(nb));
-      } else {
-        const uint32_t a = (2 * R < nval) ? __ldg(nb) : 0u, b = (2 * R + 1 < nval) ? __ldg(nb + 1) : 0u;
-        r.kn[0] = a | (b << 16);
-      }
-    } else {
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-        r.kn[rr] = (FULL || 2 * R + rr < nval) ? __ldg(reinterpret_cast<const uint32_t*>(nb + rr * NB)) : 0u;
-    }
   }
   if constexpr (LOADV) {
-    const uint8_t* base = u.vc + (size_t)t0 * NB * Fmt<VB>::kBlockBytes;
 #pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-      const bool ok = FULL || (vtok(g, tt) < nval);
+    for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        if (ok) {
-          load_vwords<VB>(r.v[tt][blk], base + lo.v[tt] + blk * Fmt<VB>::kBlockBytes, lo.vsh);
+        const int toff = ((tt & 1) << 1) + (tt >> 1);  // vtok(g, tt) - 4g
+        const uint8_t* s = vs + (toff * NB + blk) * Fmt<VB>::kBlockBytes;
+        if constexpr (VB == 4) {
+          const uint2 x = *reinterpret_cast<const uint2*>(s);
+          r.v[tt][blk][0] = x.x; r.v[tt][blk][1] = x.y;
+        } else if constexpr (VB == 3) {
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(s);
+          const uint32_t w0 = w[0], w1 = w[1];
+          if (R & 1) {
+            r.v[tt][blk][0] = __funnelshift_r(w0, w1, 16);
+            r.v[tt][blk][1] = w1 >> 16;
+          } else {
+            r.v[tt][blk][0] = w0;
+            r.v[tt][blk][1] = w1;
+          }
         } else {
-          r.v[tt][blk][0] = r.v[tt][blk][1] = 0u;
+          r.v[tt][blk][0] = *reinterpret_cast<const uint32_t*>(s);
+          r.v[tt][blk][1] = 0u;
         }
       }
-    }
-    const uint16_t* nb = u.vn + (size_t)(t0 + 2 * R) * NB;
-    if constexpr (NB == 1) {
-      if (FULL) {
-        r.vn[0] = __ldg(reinterpret_cast<const uint32_t*>(nb));
-      } else {
-        const uint32_t a = (2 * R < nval) ? __ldg(nb) : 0u, b = (2 * R + 1 < nval) ? __ldg(nb + 1) : 0u;
-        r.vn[0] = a | (b << 16);
-      }
-    } else {
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-        r.vn[rr] = (FULL || 2 * R + rr < nval) ? __ldg(reinterpret_cast<const uint32_t*>(nb + rr * NB)) : 0u;
-    }
   }
 }
 
-template <int KB, int VB, int NB, bool LOADK, bool LOADV>
-__device__ __forceinline__ void load_tile_any(TileRegs<KB, VB, NB>& r, const UnitPtrs& u,
-                                              const LaneOffsets<KB, VB, NB>& lo, int t0, int lane) {
-  if (t0 + kTile <= u.len)
-    load_tile<KB, VB, NB, LOADK, LOADV, true>(r, u, lo, t0, lane);
-  else
-    load_tile<KB, VB, NB, LOADK, LOADV, false>(r, u, lo, t0, lane);
+// Norm words of tokens 2R and 2R+1 from a ring slot (see TileRegs).
+template <int NB>
+__device__ __forceinline__ void read_norms(uint32_t (&dst)[NB], const uint8_t* nbase, int R) {
+  if constexpr (NB == 1) {
+    dst[0] = *reinterpret_cast<const uint32_t*>(nbase + 4 * R);
+  } else {
+    const uint2 x = *reinterpret_cast<const uint2*>(nbase + 8 * R);
+    dst[0] = x.x;
+    dst[1] = x.y;
+  }
 }
 
 // Norms of tokens 2R (x) and 2R+1 (y) for block blk, as fp32.
@@ -274,22 +236,6 @@ __device__ __forceinline__ float2 norm_pair(const uint32_t (&w)[NB], int blk) {
     const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&w[0]));
     const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&w[1]));
     return blk == 0 ? make_float2(a.x, b.x) : make_float2(a.y, b.y);
-  }
-}
-
-// L2 prefetch of the tokens [tok_lo, tok_hi) of one unit (one thread).
-template <int KB, int VB, int NB, bool PK, bool PV>
-__device__ __forceinline__ void prefetch_range(const UnitPtrs& u, int tok_lo, int tok_hi) {
-  if (tok_hi <= tok_lo) return;
-  const int n = tok_hi - tok_lo;
-  if constexpr (PK) prefetch_l2(u.kc + (size_t)tok_lo * NB * Fmt<KB>::kBlockBytes, n * NB * Fmt<KB>::kBlockBytes);
-  if constexpr (PV) prefetch_l2(u.vc + (size_t)tok_lo * NB * Fmt<VB>::kBlockBytes, n * NB * Fmt<VB>::kBlockBytes);
-  const int nn = (n * NB * 2) & ~15;  // norm bytes, whole 16-byte units
-  if (nn > 0) {
-    const uint16_t* a = u.kn + (size_t)tok_lo * NB;
-    const uint16_t* b = u.vn + (size_t)tok_lo * NB;
-    if (PK && (reinterpret_cast<uintptr_t>(a) & 15) == 0) prefetch_l2(a, nn);
-    if (PV && (reinterpret_cast<uintptr_t>(b) & 15) == 0) prefetch_l2(b, nn);
   }
 }
 
@@ -307,30 +253,40 @@ struct Smem {
   static constexpr bool kStaticLut = kLutK + kLutV <= kStaticLutLimit;
   static constexpr int kStaticBytes = kStaticLut ? kLutK + kLutV : 16;
   static constexpr int kDynLut = kStaticLut ? 0 : kLutK + kLutV;
-  static constexpr int kWorkFloats = kWarps * kMaxGroup * D;     // per-warp partials / qhat
+  // One ring slot holds one tile: K codes, V codes, K norms, V norms.
+  static constexpr int kSlotK = kHasK ? kTile * NB * Fmt<KB>::kBlockBytes : 0;
+  static constexpr int kSlotV = kHasV ? kTile * NB * Fmt<VB>::kBlockBytes : 0;
+  static constexpr int kSlotKN = kHasK ? kTile * NB * 2 : 0;
+  static constexpr int kSlotVN = kHasV ? kTile * NB * 2 : 0;
+  static constexpr int kOffSlotV = kSlotK;
+  static constexpr int kOffSlotKN = kOffSlotV + kSlotV;
+  static constexpr int kOffSlotVN = kOffSlotKN + kSlotKN;
+  static constexpr int kSlotBytes = (kOffSlotVN + kSlotVN + 127) / 128 * 128;
+  static constexpr int kWorkFloats = kCWarps * kMaxGroup * D;    // per-warp partials / qhat
   static constexpr int kResFloats = kMaxGroup * D;               // merged rotated-domain acc
   static constexpr int kOffLutK = 0;
   static constexpr int kOffLutV = kOffLutK + kLutK;
-  static constexpr int kOffDyn = kDynLut;
-  static constexpr int kOffWork = kOffDyn;
+  static constexpr int kOffRing = (kDynLut + 127) / 128 * 128;
+  static constexpr int kOffWork = kOffRing + kCWarps * kDepth * kSlotBytes;
   static constexpr int kOffRes = kOffWork + kWorkFloats * 4;
   static constexpr int kOffMisc = kOffRes + kResFloats * 4;
-  // misc: warp m/l [kWarps][8] x2, merged M/L/lse [8] x3, qexp [8], flag, then batch prefix.
-  static constexpr int kMiscFloats = 2 * kWarps * kMaxGroup + 4 * kMaxGroup + 4 + 2 * kThreads +
-                                     kMergeChunk * kMaxGroup;
+  // misc: warp m/l [kCWarps][8] x2, merged M/L/lse [8] x3, qexp [8], warp
+  // totals [16], flags [4], reduction scratch [kCThreads] x2, merge factors.
+  static constexpr int kMiscFloats = 2 * kCWarps * kMaxGroup + 4 * kMaxGroup + 16 + 4 +
+                                     2 * kCThreads + kMergeChunk * kMaxGroup;
   static constexpr int kOffPrefix = kOffMisc + kMiscFloats * 4;
   static size_t bytes(int batch) { return (size_t)kOffPrefix + (size_t)(batch + 1) * 4; }
 };
 
 // Per-head (M, L) = (max m, sum l * 2^(m - M)) over the partials of one unit,
-// using every thread: thread t takes head t % 8 and every (kThreads/8)-th
-// partial, folding them in a fixed order; the kThreads/8 running pairs of a
-// head are then combined in a fixed order.  Partials of CTAs whose range is
-// empty are skipped.
+// using every consumer thread: thread t takes head t % 8 and every
+// (kCThreads/8)-th partial, folding them in a fixed order; the running pairs
+// of a head are then combined in a fixed order.  Partials of CTAs whose range
+// is empty are skipped.
 __device__ __forceinline__ void unit_stats(const float* slot_ml, long long c_first, long long c_last,
                                            long long parts, long long T, long long unit, int Gu,
                                            float* red_m, float* red_l, float* outM, float* outL) {
-  constexpr int J = kThreads / kMaxGroup;
+  constexpr int J = kCThreads / kMaxGroup;
   const int tid = threadIdx.x, hd = tid % kMaxGroup, j = tid / kMaxGroup;
   float m = -INFINITY, l = 0.0f;
   if (hd < Gu) {
@@ -349,7 +305,7 @@ __device__ __forceinline__ void unit_stats(const float* slot_ml, long long c_fir
   }
   red_m[tid] = m;
   red_l[tid] = l;
-  __syncthreads();
+  consumer_sync();
   if (tid < Gu) {
     float M = -INFINITY;
     for (int jj = 0; jj < J; ++jj) M = fmaxf(M, red_m[jj * kMaxGroup + tid]);
@@ -361,7 +317,39 @@ __device__ __forceinline__ void unit_stats(const float* slot_ml, long long c_fir
     outM[tid] = M;
     outL[tid] = L;
   }
-  __syncthreads();
+  consumer_sync();
+}
+
+// Where tile x of the flattened (unit, tile) space lies.
+struct Segment {
+  int b, r, nt, unit, kvh, hg, h0, Gu, len, seg_lo, seg_hi;
+  long long Su;
+};
+
+__device__ __forceinline__ Segment locate(long long x, long long hi, const int* prefix, int batch,
+                                          int UB, int n_hg, int G, int seq_cap,
+                                          const int32_t* seq_lens) {
+  Segment s;
+  const long long y = x / UB;  // in units of "tiles per batch entry"
+  int bl = 0, bh = batch;      // largest b with prefix[b] <= y
+  while (bh - bl > 1) {
+    const int mid = (bl + bh) >> 1;
+    if (prefix[mid] <= y) bl = mid; else bh = mid;
+  }
+  s.b = bl;
+  s.nt = prefix[bl + 1] - prefix[bl];
+  const long long TB = (long long)prefix[bl] * UB;
+  s.r = (int)((x - TB) / s.nt);
+  s.Su = TB + (long long)s.r * s.nt;
+  s.seg_lo = (int)(x - s.Su);
+  s.seg_hi = (int)(min(hi, s.Su + s.nt) - s.Su);
+  s.unit = bl * UB + s.r;
+  s.kvh = s.r / n_hg;
+  s.hg = s.r % n_hg;
+  s.h0 = s.kvh * G + s.hg * kMaxGroup;
+  s.Gu = min(kMaxGroup, G - s.hg * kMaxGroup);
+  s.len = min(max(__ldg(seq_lens + bl), 0), seq_cap);
+  return s;
 }
 
 // --------------------------------------------------------------- the kernel --
@@ -372,24 +360,27 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   using SM = Smem<KB, VB, NB, MODE>;
   constexpr int D = SM::D;
   constexpr bool HASK = SM::kHasK, HASV = SM::kHasV;
+  constexpr int KBB = Fmt<KB>::kBlockBytes, VBB = Fmt<VB>::kBlockBytes;
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(128) uint8_t slut[SM::kStaticBytes];
   uint8_t* lut_base = SM::kStaticLut ? slut : smem;
   uint8_t* lutK = lut_base + SM::kOffLutK;
   uint8_t* lutV = lut_base + SM::kOffLutV;
+  uint8_t* ring = smem + SM::kOffRing;
   float* work = reinterpret_cast<float*>(smem + SM::kOffWork);
   float* res = reinterpret_cast<float*>(smem + SM::kOffRes);
   float* misc = reinterpret_cast<float*>(smem + SM::kOffMisc);
-  float* w_m = misc;                                  // [kWarps][8]
-  float* w_l = misc + kWarps * kMaxGroup;             // [kWarps][8]
-  float* u_M = misc + 2 * kWarps * kMaxGroup;         // [8]
+  float* w_m = misc;                                  // [kCWarps][8]
+  float* w_l = misc + kCWarps * kMaxGroup;            // [kCWarps][8]
+  float* u_M = misc + 2 * kCWarps * kMaxGroup;        // [8]
   float* u_L = u_M + kMaxGroup;                       // [8]
   float* u_lse = u_L + kMaxGroup;                     // [8]
   int* qexp = reinterpret_cast<int*>(u_lse + kMaxGroup);  // [8]
-  int* flag = qexp + kMaxGroup;
-  float* red_m = reinterpret_cast<float*>(flag + 4);  // [kThreads]
-  float* red_l = red_m + kThreads;                     // [kThreads]
-  float* fac = red_l + kThreads;                       // [kMergeChunk][8]
+  int* wtot = qexp + kMaxGroup;                       // [16]
+  int* flag = wtot + 16;                              // [4]
+  float* red_m = reinterpret_cast<float*>(flag + 4);  // [kCThreads]
+  float* red_l = red_m + kCThreads;                   // [kCThreads]
+  float* fac = red_l + kCThreads;                     // [kMergeChunk][8]
   int* prefix = reinterpret_cast<int*>(smem + SM::kOffPrefix);  // [B+1] tiles per batch, prefix
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -429,17 +420,16 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       }
       local += (len + kTile - 1) / kTile;
     }
-    // block-wide exclusive scan of `local`
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    if (lane == 31) qexp[warp] = incl;  // temporary use of qexp as warp totals
+    if (lane == 31) wtot[warp] = incl;
     __syncthreads();
     int warp_off = 0;
-    for (int w = 0; w < warp; ++w) warp_off += qexp[w];
+    for (int w = 0; w < warp; ++w) warp_off += wtot[w];
     int run = warp_off + incl - local;
     for (int b = b_lo; b < min(B, b_lo + per); ++b) {
       prefix[b] = run;
@@ -467,44 +457,27 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   const long long lo = (long long)blockIdx.x * T / P;
   const long long hi = ((long long)blockIdx.x + 1) * T / P;
   auto cta_of = [&](long long x, long long parts) { return ((x + 1) * parts + T - 1) / T - 1; };
-
-  long long x = lo;
-  while (x < hi) {
-    // ---- locate the unit holding tile x ------------------------------------
-    const long long y = x / UB;  // in units of "tiles per batch entry"
-    int bl = 0, bh = p.batch;    // largest b with prefix[b] <= y
-    while (bh - bl > 1) {
-      const int mid = (bl + bh) >> 1;
-      if (prefix[mid] <= y) bl = mid; else bh = mid;
-    }
-    const int b = bl;
-    const int nt = prefix[b + 1] - prefix[b];
-    const long long TB = (long long)prefix[b] * UB;
-    const int r = (int)((x - TB) / nt);
-    const long long Su = TB + (long long)r * nt;
-    const int seg_lo = (int)(x - Su);
-    const int seg_hi = (int)(min(hi, Su + nt) - Su);
-    const int unit = b * UB + r;
-    const int kvh = r / n_hg, hg = r % n_hg;
-    const int h0 = kvh * G + hg * kMaxGroup;
-    const int Gu = min(kMaxGroup, G - hg * kMaxGroup);
-    const int len = min(max(__ldg(p.seq_lens + b), 0), p.seq_cap);
-
-    UnitPtrs up;
-    const size_t cache_row = (size_t)(b * p.kv_heads + kvh) * p.seq_cap;
-    up.kc = p.k_codes + cache_row * NB * Fmt<KB>::kBlockBytes;
-    up.kn = p.k_norms + cache_row * NB;
-    up.vc = p.v_codes + cache_row * NB * Fmt<VB>::kBlockBytes;
-    up.vn = p.v_norms + cache_row * NB;
-    up.len = len;
+  const int cw = warp;
+  uint8_t* wring = ring + (size_t)cw * kDepth * SM::kSlotBytes;  // this warp's ring
+  const uint32_t wring_s = smem_addr(wring);
+  for (long long x = lo; x < hi;) {
+    const Segment sg = locate(x, hi, prefix, p.batch, UB, n_hg, G, p.seq_cap, p.seq_lens);
+    const int b = sg.b, nt = sg.nt, unit = sg.unit, h0 = sg.h0, Gu = sg.Gu, len = sg.len;
+    const int seg_lo = sg.seg_lo, seg_hi = sg.seg_hi;
+    const long long Su = sg.Su;
+    const size_t cache_row = (size_t)(b * p.kv_heads + sg.kvh) * p.seq_cap;
+    const uint8_t* kcp = p.k_codes + cache_row * NB * KBB;
+    const uint8_t* vcp = p.v_codes + cache_row * NB * VBB;
+    const uint16_t* knp = p.k_norms + cache_row * NB;
+    const uint16_t* vnp = p.v_norms + cache_row * NB;
 
     // ---- per-unit query preparation: qhat = H.(s o q) (D1) ----------------
     uint32_t qf[NB][8][2];
-    float qmul[2];
+    float qmul[2] = {0.0f, 0.0f};
     float lse2[2] = {0.0f, 0.0f};
     if constexpr (HASK) {
       float* qs = work;  // [8][D]
-      for (int i = tid; i < kMaxGroup * D; i += kThreads) {
+      for (int i = tid; i < kMaxGroup * D; i += kCThreads) {
         const int j = i / D, d = i % D;
         float v = 0.0f;
         if (j < Gu) {
@@ -516,9 +489,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         }
         qs[i] = v;
       }
-      __syncthreads();
+      consumer_sync();
       for (int s = 1; s < kBlock; s <<= 1) {
-        for (int i = tid; i < kMaxGroup * D / 2; i += kThreads) {
+        for (int i = tid; i < kMaxGroup * D / 2; i += kCThreads) {
           const int j = i / (D / 2), rem = i % (D / 2);
           const int a = (rem / s) * 2 * s + (rem % s);
           float* row = qs + j * D;
@@ -526,18 +499,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           row[a] = u + w;
           row[a + s] = u - w;
         }
-        __syncthreads();
+        consumer_sync();
       }
       // power-of-two scale per head so fp16 fragments neither overflow nor
       // fall into subnormals
-      for (int j = warp; j < kMaxGroup; j += kWarps) {
+      for (int j = cw; j < kMaxGroup; j += kCWarps) {
         float mx = 0.0f;
         for (int d = lane; d < D; d += 32) mx = fmaxf(mx, fabsf(qs[j * D + d]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         if (lane == 0) qexp[j] = (mx > 0.0f) ? (ilogbf(mx) - 13) : 0;
       }
-      __syncthreads();
+      consumer_sync();
       const float qsc = ldexpf(1.0f, -qexp[R]);
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
@@ -550,24 +523,22 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       }
       qmul[0] = p.score_mult * ldexpf(1.0f, qexp[2 * g]);
       qmul[1] = p.score_mult * ldexpf(1.0f, qexp[2 * g + 1]);
-      __syncthreads();  // work area is reused below
+      consumer_sync();  // work area is reused below
     }
     if constexpr (MODE == kSparseV) {
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote
-      {
-        const long long P1 = p1_ctas;
-        unit_stats(p.slot_ml, cta_of(Su, P1), cta_of(Su + nt - 1, P1), P1, T, unit, Gu, red_m, red_l,
-                   u_M, u_L);
-        if (tid < Gu) u_lse[tid] = u_M[tid] + __log2f(u_L[tid]);
-        __syncthreads();
-      }
+      const long long P1 = p1_ctas;
+      unit_stats(p.slot_ml, cta_of(Su, P1), cta_of(Su + nt - 1, P1), P1, T, unit, Gu, red_m, red_l,
+                 u_M, u_L);
+      if (tid < Gu) u_lse[tid] = u_M[tid] + __log2f(u_L[tid]);
+      consumer_sync();
       lse2[0] = (2 * g < Gu) ? u_lse[2 * g] : 0.0f;
       lse2[1] = (2 * g + 1 < Gu) ? u_lse[2 * g + 1] : 0.0f;
     }
     const float log2_thr = (MODE == kSparseV) ? __log2f(p.sparse_thr) : 0.0f;
 
-    // ---- warp loop over this segment's tiles ------------------------------
+    // ---- warp loop over this segment's stages -----------------------------
     float acc[NB][8][4];
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk)
@@ -578,7 +549,6 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.0f, 0.0f};
 
-    const LaneOffsets<KB, VB, NB> loff(lane);
     auto compute = [&](const TileRegs<KB, VB, NB>& tr, int tile) {
       const int t0 = tile * kTile;
       // rows R and R+8 of the score tile are tokens 2R and 2R+1
@@ -712,34 +682,83 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     };
 
     {
-      // Warp w takes tiles seg_lo + w, seg_lo + w + kWarps, ...; one thread
-      // keeps the L2 kPrefetchSteps tile groups ahead of the CTA.
-      const bool pf_thread = (tid == 0);
-      auto prefetch_group = [&](int first_tile) {
-        const int a = max(first_tile, seg_lo), e = min(first_tile + kWarps, seg_hi);
-        if (a < e) prefetch_range<KB, VB, NB, HASK, HASV>(up, a * kTile, min(e * kTile, len));
+      // Copy tile `tile` of this unit into ring slot `slot` (all lanes; one
+      // commit group).  Bytes past the end of the sequence are zero-filled.
+      auto issue = [&](int tile, int slot) {
+        const int t0 = tile * kTile;
+        const int nval = min(kTile, len - t0);  // >= 1
+        const uint32_t sb = wring_s + (uint32_t)(slot * SM::kSlotBytes);
+        if constexpr (HASK) {
+          constexpr int kChunks = kTile * NB * KB;  // 16-byte chunks (KBB = 16 * KB)
+          constexpr int kPerTok = NB * KB;
+          const uint8_t* src = kcp + (size_t)t0 * NB * KBB;
+#pragma unroll
+          for (int c0 = 0; c0 < kChunks; c0 += 32) {
+            const int c = c0 + lane;
+            if (c < kChunks) {
+              const bool ok = c / kPerTok < nval;
+              cp_async16(sb + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
+            }
+          }
+          if (lane < 8 * NB) {  // norms: 4-byte pieces of the tile's 16*NB halves
+            const int e = 2 * lane;  // first half of the piece
+            const int valid = max(0, min(2, nval * NB - e));
+            cp_async4(sb + SM::kOffSlotKN + 4u * lane, knp + (size_t)t0 * NB + (valid ? e : 0),
+                      2u * (uint32_t)valid);
+          }
+        }
+        if constexpr (HASV) {
+          constexpr int kChunks = kTile * NB * VB;
+          constexpr int kPerTok = NB * VB;
+          const uint8_t* src = vcp + (size_t)t0 * NB * VBB;
+#pragma unroll
+          for (int c0 = 0; c0 < kChunks; c0 += 32) {
+            const int c = c0 + lane;
+            if (c < kChunks) {
+              const bool ok = c / kPerTok < nval;
+              cp_async16(sb + SM::kOffSlotV + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
+            }
+          }
+          if (lane < 8 * NB) {
+            const int e = 2 * lane;
+            const int valid = max(0, min(2, nval * NB - e));
+            cp_async4(sb + SM::kOffSlotVN + 4u * lane, vnp + (size_t)t0 * NB + (valid ? e : 0),
+                      2u * (uint32_t)valid);
+          }
+        }
       };
-      if (pf_thread)
-        prefetch_range<KB, VB, NB, HASK, HASV>(up, seg_lo * kTile,
-                                               min(min(seg_hi, seg_lo + (kPrefetchSteps + 1) * kWarps) * kTile, len));
-      TileRegs<KB, VB, NB> ta, tb;
-      int k = seg_lo + warp;
-      int step = 0;
-      if (k < seg_hi) load_tile_any<KB, VB, NB, HASK, HASV>(ta, up, loff, k * kTile, lane);
-      for (;;) {
-        if (k >= seg_hi) break;
-        if (k + kWarps < seg_hi) load_tile_any<KB, VB, NB, HASK, HASV>(tb, up, loff, (k + kWarps) * kTile, lane);
-        if (pf_thread) prefetch_group(seg_lo + (step + kPrefetchSteps + 1) * kWarps);
-        compute(ta, k);
-        k += kWarps;
-        ++step;
-        if (k >= seg_hi) break;
-        if (k + kWarps < seg_hi) load_tile_any<KB, VB, NB, HASK, HASV>(ta, up, loff, (k + kWarps) * kTile, lane);
-        if (pf_thread) prefetch_group(seg_lo + (step + kPrefetchSteps + 1) * kWarps);
-        compute(tb, k);
-        k += kWarps;
-        ++step;
+
+      // This lane's first K / V word inside a slot.
+      const int vlane = VB == 4 ? 8 * R : (VB == 3 ? 4 * ((3 * R) >> 1) : 4 * R);
+      const uint32_t koff = (uint32_t)((2 * R) * NB * KBB + g * KB * 4);
+      const uint32_t voff = (uint32_t)(SM::kOffSlotV + (4 * g) * NB * VBB + vlane);
+      // Warp cw takes tiles seg_lo + cw, seg_lo + cw + kCWarps, ...: tile i of
+      // the warp (i = 0, 1, ...) lives in slot i % kDepth.
+      const int first = seg_lo + cw;
+      const int n_mine = first < seg_hi ? (seg_hi - first + kCWarps - 1) / kCWarps : 0;
+#pragma unroll
+      for (int i = 0; i < kDepth - 1; ++i) {
+        if (i < n_mine) issue(first + i * kCWarps, i);
+        cp_async_commit();
       }
+      for (int i = 0; i < n_mine; ++i) {
+        const int tile = first + i * kCWarps;
+        const int slot = i % kDepth;
+        cp_async_wait<kDepth - 2>();  // this warp's copies of tile i have landed
+        __syncwarp();
+        TileRegs<KB, VB, NB> tr;
+        const uint8_t* sl = wring + (size_t)slot * SM::kSlotBytes;
+        read_tile<KB, VB, NB, HASK, HASV>(tr, sl + koff, sl + voff, R);
+        if constexpr (HASK) read_norms<NB>(tr.kn, sl + SM::kOffSlotKN, R);
+        if constexpr (HASV) read_norms<NB>(tr.vn, sl + SM::kOffSlotVN, R);
+        compute(tr, tile);
+        // refill: tile i + kDepth - 1 goes to the slot freed by tile i - 1
+        __syncwarp();
+        if (i + kDepth - 1 < n_mine) issue(first + (i + kDepth - 1) * kCWarps, (i + kDepth - 1) % kDepth);
+        cp_async_commit();
+      }
+      cp_async_wait<0>();
+      __syncwarp();
     }
 
     // ---- warp partials to shared memory -----------------------------------
@@ -750,8 +769,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       if (R == 0) {
-        w_m[warp * kMaxGroup + 2 * g + cc] = m_run[cc];
-        w_l[warp * kMaxGroup + 2 * g + cc] = l;
+        w_m[cw * kMaxGroup + 2 * g + cc] = m_run[cc];
+        w_l[cw * kMaxGroup + 2 * g + cc] = l;
       }
     }
     if constexpr (HASV) {
@@ -760,21 +779,21 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
           const int d0 = blk * kBlock + 16 * R + 2 * mt;
-          float* w0 = work + (warp * kMaxGroup + 2 * g) * D + d0;
-          float* w1 = work + (warp * kMaxGroup + 2 * g + 1) * D + d0;
+          float* w0 = work + (cw * kMaxGroup + 2 * g) * D + d0;
+          float* w1 = work + (cw * kMaxGroup + 2 * g + 1) * D + d0;
           *reinterpret_cast<float2*>(w0) = make_float2(acc[blk][mt][0], acc[blk][mt][2]);
           *reinterpret_cast<float2*>(w1) = make_float2(acc[blk][mt][1], acc[blk][mt][3]);
         }
     }
-    __syncthreads();
+    consumer_sync();
 
     // ---- merge the warps in a fixed order ----------------------------------
     if constexpr (HASK) {
       if (tid < Gu) {
         float M = -INFINITY;
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, w_m[w * kMaxGroup + tid]);
+        for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, w_m[w * kMaxGroup + tid]);
         float L = 0.0f;
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < kCWarps; ++w) {
           const float mw = w_m[w * kMaxGroup + tid];
           if (mw != -INFINITY) L += w_l[w * kMaxGroup + tid] * ex2(mw - M);
         }
@@ -783,15 +802,15 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       }
     }
     if constexpr (HASV) {
-      for (int i = tid; i < Gu * D; i += kThreads) {
+      for (int i = tid; i < Gu * D; i += kCThreads) {
         const int hd = i / D, d = i % D;
         float M = 0.0f;
         if constexpr (HASK) {
           M = -INFINITY;
-          for (int w = 0; w < kWarps; ++w) M = fmaxf(M, w_m[w * kMaxGroup + hd]);
+          for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, w_m[w * kMaxGroup + hd]);
         }
         float s = 0.0f;
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < kCWarps; ++w) {
           float f = 1.0f;
           if constexpr (HASK) {
             const float mw = w_m[w * kMaxGroup + hd];
@@ -802,7 +821,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         res[i] = s;
       }
     }
-    __syncthreads();
+    consumer_sync();
 
     const bool whole = (seg_lo == 0 && seg_hi == nt);
     bool finalize = false;
@@ -818,27 +837,27 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         }
       }
       if constexpr (HASV) {
-        for (int i = tid; i < Gu * D; i += kThreads)
+        for (int i = tid; i < Gu * D; i += kCThreads)
           p.slot_acc[(slot * kMaxGroup + i / D) * D + i % D] = res[i];
       }
       if constexpr (MODE != kScores) {
         __threadfence();
-        __syncthreads();
+        consumer_sync();
         if (tid == 0) {
           const unsigned add = (unsigned)(seg_hi - seg_lo);
           const unsigned old = atomicAdd(p.tickets + unit, add);
           flag[0] = (old + add == (unsigned)nt) ? 1 : 0;
         }
-        __syncthreads();
+        consumer_sync();
         finalize = flag[0] != 0;
         if (finalize) {
           __threadfence();
           const long long c_first = cta_of(Su, P), c_last = cta_of(Su + nt - 1, P);
           if constexpr (HASK) unit_stats(p.slot_ml, c_first, c_last, P, T, unit, Gu, red_m, red_l, u_M, u_L);
-          for (int i = tid; i < Gu * D; i += kThreads) res[i] = 0.0f;
+          for (int i = tid; i < Gu * D; i += kCThreads) res[i] = 0.0f;
           for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
             // weights 2^(m_c - M) of this chunk's partials (0 for empty ranges)
-            for (int i = tid; i < kMergeChunk * kMaxGroup; i += kThreads) {
+            for (int i = tid; i < kMergeChunk * kMaxGroup; i += kCThreads) {
               const long long c = c0 + i / kMaxGroup;
               const int hd = i % kMaxGroup;
               float f = 0.0f;
@@ -851,9 +870,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
               }
               fac[i] = f;
             }
-            __syncthreads();
+            consumer_sync();
             const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
-            for (int i = tid; i < Gu * D; i += kThreads) {
+            for (int i = tid; i < Gu * D; i += kCThreads) {
               const int hd = i / D, d = i % D;
               const float* src = p.slot_acc + ((c0 + unit) * kMaxGroup + hd) * D + d;
               float sacc = res[i];
@@ -865,10 +884,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
               }
               res[i] = sacc;
             }
-            __syncthreads();
+            consumer_sync();
           }
           if (tid == 0) p.tickets[unit] = 0u;
-          __syncthreads();
+          consumer_sync();
         }
       }
     }
@@ -876,7 +895,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     if (finalize) {
       // ---- D7/D8: one inverse rotation per head, o = s o (H.acc) / L -----
       for (int s = 1; s < kBlock; s <<= 1) {
-        for (int i = tid; i < Gu * D / 2; i += kThreads) {
+        for (int i = tid; i < Gu * D / 2; i += kCThreads) {
           const int hd = i / (D / 2), rem = i % (D / 2);
           const int a = (rem / s) * 2 * s + (rem % s);
           float* row = res + hd * D;
@@ -884,9 +903,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           row[a] = u + w;
           row[a + s] = u - w;
         }
-        __syncthreads();
+        consumer_sync();
       }
-      for (int i = tid; i < Gu * D; i += kThreads) {
+      for (int i = tid; i < Gu * D; i += kCThreads) {
         const int hd = i / D, d = i % D;
         const int e = d & (kBlock - 1);
         float v = res[i];
@@ -895,7 +914,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         p.out[((size_t)b * p.q_heads + h0 + hd) * D + d] = v;
       }
     }
-    __syncthreads();
+    consumer_sync();
     x = Su + seg_hi;
   }
 }

@@ -222,6 +222,7 @@ int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const t
   int st = check_desc(desc);
   if (st != TQ_OK) return st;
   if (desc->batch > tq::kMaxBatch || desc->head_dim > tq::kMaxDecodeHeadDim) return TQ_ERR_UNSUPPORTED;
+  if (desc->seq_cap % 2 != 0) return TQ_ERR_UNSUPPORTED;  // norm rows must start 4-byte aligned
   if ((long long)desc->batch * ((desc->seq_cap + tq::kTile - 1) / tq::kTile) >= (1LL << 31))
     return TQ_ERR_UNSUPPORTED;
   if (q_heads < desc->kv_heads || q_heads % desc->kv_heads != 0) return TQ_ERR_INVALID_ARG;

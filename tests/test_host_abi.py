@@ -134,6 +134,10 @@ def test_decode_rejects_bad_arguments_without_launch():
     # sparse mode needs the score buffer: the dense size is too small
     assert call(thr=1e-5) == _lib.TQ_ERR_WORKSPACE
     assert call(desc=tq.kv_desc(2, 2, 384, 64, 3, 2)) in (_lib.TQ_ERR_UNSUPPORTED, _lib.TQ_ERR_WORKSPACE)
+    odd = tq.kv_desc(2, 2, 128, 63, 3, 2)
+    assert lib.tq_decode_attention(ctypes.byref(odd), ctypes.byref(cb3), ctypes.byref(cb2), 8, _fake(GOOD), 1,
+                                   _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), 0.1, 0.0,
+                                   _fake(GOOD), _fake(GOOD), 1 << 30, None, None) == _lib.TQ_ERR_UNSUPPORTED
 
 
 def test_workspace_size_formula():
