@@ -36,6 +36,8 @@
 
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "../../include/tq.h"
 #include "tq_internal.h"
 
@@ -77,7 +79,7 @@ __device__ __forceinline__ uint32_t movtrans(uint32_t x) {
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -97,22 +99,67 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// Byte offset into a lane-replicated table: field of `fb` bits at bit `pos`
-// of the word array w, times 128 (32 lanes x 4 bytes per entry), plus lane*4.
-// Called with compile-time pos/fb after unrolling, so the branches fold.
-__device__ __forceinline__ uint32_t lut_off(const uint32_t* w, int pos, int fb, uint32_t lane4) {
-  const int wi = pos >> 5, sh = pos & 31;
-  const uint32_t mask = ((1u << fb) - 1u) << 7;
-  uint32_t v;
-  if (sh + fb <= 32)
-    v = (sh >= 7) ? (w[wi] >> (sh - 7)) : (w[wi] << (7 - sh));
-  else
-    v = __funnelshift_r(w[wi], w[wi + 1], sh) << 7;
-  return (v & mask) | lane4;
+// Shared-memory loads on 32-bit shared-window addresses (volatile: they are
+// ordered with the asynchronous copies and barriers around them).
+__device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
+  uint32_t x;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(x) : "r"(a));
+  return x;
+}
+__device__ __forceinline__ uint2 ld_s64(uint32_t a) {
+  uint2 x;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(x.x), "=r"(x.y) : "r"(a));
+  return x;
+}
+__device__ __forceinline__ uint4 ld_s128(uint32_t a) {
+  uint4 x;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(a));
+  return x;
 }
 
-__device__ __forceinline__ uint32_t lds(const uint8_t* base, uint32_t off) {
-  return *reinterpret_cast<const uint32_t*>(base + off);
+// Table read.  Not volatile: the tables do not change after the prologue, and
+// every address depends on code words read (volatile, after the copy waits)
+// from the ring, so the compiler may schedule these freely, e.g. ahead of the
+// softmax that precedes their use.
+__device__ __forceinline__ uint32_t ld_table(uint32_t a) {
+  uint32_t x;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(x) : "r"(a));
+  return x;
+}
+
+// Lane-replicated table lookup.  The table holds, for every value of a field
+// of `fb` bits (two codes), one 4-byte entry per lane: entry f of lane l sits
+// at table + f*128 + l*4, so the 32 lanes always hit 32 different banks.
+// `lb` is table + lane*4.  When the table is aligned to its own size the
+// field bits can be OR-ed into lb (ALIGNED); otherwise they are added.  The
+// field is the one at bit `pos` of the word array w; pos and fb are
+// compile-time after unrolling, so exactly one of the forms below is emitted:
+// a shift and one three-input logic op (plus an add when not ALIGNED), or a
+// funnel shift for a field that crosses a word boundary.
+template <bool ALIGNED>
+__device__ __forceinline__ uint32_t lut_get(const uint32_t* w, int pos, int fb, uint32_t lb) {
+  const int wi = pos >> 5, sh = pos & 31;
+  const uint32_t mask = ((1u << fb) - 1u) << 7;
+  uint32_t a;
+  if (sh + fb > 32) {
+    const uint32_t v = __funnelshift_r(w[wi], w[wi + 1], sh) << 7;
+    a = ALIGNED ? ((v & mask) | lb) : ((v & mask) + lb);
+  } else if (sh >= 7) {
+    if (ALIGNED)
+      asm("{ .reg .b32 t; shr.b32 t, %1, %2; and.b32 t, t, %3; or.b32 %0, t, %4; }"
+          : "=r"(a) : "r"(w[wi]), "r"(sh - 7), "r"(mask), "r"(lb));
+    else
+      asm("{ .reg .b32 t; shr.b32 t, %1, %2; and.b32 t, t, %3; add.u32 %0, t, %4; }"
+          : "=r"(a) : "r"(w[wi]), "r"(sh - 7), "r"(mask), "r"(lb));
+  } else {
+    if (ALIGNED)
+      asm("{ .reg .b32 t; shl.b32 t, %1, %2; and.b32 t, t, %3; or.b32 %0, t, %4; }"
+          : "=r"(a) : "r"(w[wi]), "r"(7 - sh), "r"(mask), "r"(lb));
+    else
+      asm("{ .reg .b32 t; shl.b32 t, %1, %2; and.b32 t, t, %3; add.u32 %0, t, %4; }"
+          : "=r"(a) : "r"(w[wi]), "r"(7 - sh), "r"(mask), "r"(lb));
+  }
+  return ld_table(a);
 }
 
 // ---------------------------------------------------------- async copies --
@@ -164,51 +211,44 @@ struct TileRegs {
   uint32_t vn[NB];
 };
 
-// Code words of one tile from a ring stage.  ks / vs point at this lane's
-// first K / V word of the warp's tile (see the lane offsets in the kernel).
+// Code words of one tile from a ring slot.  ks / vs are the shared addresses
+// of this lane's first K / V word in the slot.
 template <int KB, int VB, int NB, bool LOADK, bool LOADV>
-__device__ __forceinline__ void read_tile(TileRegs<KB, VB, NB>& r, const uint8_t* ks, const uint8_t* vs,
-                                          int R) {
+__device__ __forceinline__ void read_tile(TileRegs<KB, VB, NB>& r, uint32_t ks, uint32_t vs, int R) {
   if constexpr (LOADK) {
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        const uint8_t* s = ks + (rr * NB + blk) * Fmt<KB>::kBlockBytes;
+        const uint32_t s = ks + (rr * NB + blk) * Fmt<KB>::kBlockBytes;
         if constexpr (KB == 4) {
-          const uint4 x = *reinterpret_cast<const uint4*>(s);
+          const uint4 x = ld_s128(s);
           r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y; r.k[rr][blk][2] = x.z; r.k[rr][blk][3] = x.w;
         } else if constexpr (KB == 3) {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(s);
-          r.k[rr][blk][0] = w[0]; r.k[rr][blk][1] = w[1]; r.k[rr][blk][2] = w[2];
+          r.k[rr][blk][0] = ld_s32(s); r.k[rr][blk][1] = ld_s32(s + 4); r.k[rr][blk][2] = ld_s32(s + 8);
         } else {
-          const uint2 x = *reinterpret_cast<const uint2*>(s);
+          const uint2 x = ld_s64(s);
           r.k[rr][blk][0] = x.x; r.k[rr][blk][1] = x.y;
         }
       }
   }
   if constexpr (LOADV) {
+    const uint32_t vsh = (VB == 3 && (R & 1)) ? 16u : 0u;
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
         const int toff = ((tt & 1) << 1) + (tt >> 1);  // vtok(g, tt) - 4g
-        const uint8_t* s = vs + (toff * NB + blk) * Fmt<VB>::kBlockBytes;
+        const uint32_t s = vs + (toff * NB + blk) * Fmt<VB>::kBlockBytes;
         if constexpr (VB == 4) {
-          const uint2 x = *reinterpret_cast<const uint2*>(s);
+          const uint2 x = ld_s64(s);
           r.v[tt][blk][0] = x.x; r.v[tt][blk][1] = x.y;
         } else if constexpr (VB == 3) {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(s);
-          const uint32_t w0 = w[0], w1 = w[1];
-          if (R & 1) {
-            r.v[tt][blk][0] = __funnelshift_r(w0, w1, 16);
-            r.v[tt][blk][1] = w1 >> 16;
-          } else {
-            r.v[tt][blk][0] = w0;
-            r.v[tt][blk][1] = w1;
-          }
+          const uint32_t w0 = ld_s32(s), w1 = ld_s32(s + 4);
+          r.v[tt][blk][0] = __funnelshift_r(w0, w1, vsh);
+          r.v[tt][blk][1] = w1 >> vsh;
         } else {
-          r.v[tt][blk][0] = *reinterpret_cast<const uint32_t*>(s);
+          r.v[tt][blk][0] = ld_s32(s);
           r.v[tt][blk][1] = 0u;
         }
       }
@@ -217,11 +257,11 @@ __device__ __forceinline__ void read_tile(TileRegs<KB, VB, NB>& r, const uint8_t
 
 // Norm words of tokens 2R and 2R+1 from a ring slot (see TileRegs).
 template <int NB>
-__device__ __forceinline__ void read_norms(uint32_t (&dst)[NB], const uint8_t* nbase, int R) {
+__device__ __forceinline__ void read_norms(uint32_t (&dst)[NB], uint32_t nbase, int R) {
   if constexpr (NB == 1) {
-    dst[0] = *reinterpret_cast<const uint32_t*>(nbase + 4 * R);
+    dst[0] = ld_s32(nbase + 4 * R);
   } else {
-    const uint2 x = *reinterpret_cast<const uint2*>(nbase + 8 * R);
+    const uint2 x = ld_s64(nbase + 8 * R);
     dst[0] = x.x;
     dst[1] = x.y;
   }
@@ -248,11 +288,21 @@ struct Smem {
   static constexpr bool kHasV = MODE != kScores;
   static constexpr int kLutK = kHasK ? Fmt<KB>::kLutBytes : 0;
   static constexpr int kLutV = kHasV ? Fmt<VB>::kLutBytes : 0;
-  // Tables that fit live in static shared memory (their base then folds into
-  // the load's immediate offset); larger ones go to dynamic shared memory.
-  static constexpr bool kStaticLut = kLutK + kLutV <= kStaticLutLimit;
-  static constexpr int kStaticBytes = kStaticLut ? kLutK + kLutV : 16;
-  static constexpr int kDynLut = kStaticLut ? 0 : kLutK + kLutV;
+  // Tables of up to 8 KB live in static shared memory with room to place them
+  // at an address aligned to their own size (field bits then OR into the
+  // address); a larger table lives unaligned in dynamic shared memory.
+  static constexpr bool kAlignK = kLutK <= 8192;
+  static constexpr bool kAlignV = kLutV <= 8192;
+  // Both aligned tables share one static array: the larger one first, at an
+  // address aligned to its size; the smaller follows (still aligned, since
+  // the sizes are powers of two).  Slack: the larger size.
+  static constexpr int kAK = (kAlignK && kLutK) ? kLutK : 0;
+  static constexpr int kAV = (kAlignV && kLutV) ? kLutV : 0;
+  static constexpr int kAMax = kAK > kAV ? kAK : kAV;
+  static constexpr int kRawLut = (kAK + kAV) ? kAK + kAV + kAMax : 16;
+  static constexpr bool kKFirst = kAK >= kAV;
+  static constexpr bool kStaticLut = false;  // unaligned tables, if any, are dynamic
+  static constexpr int kDynLut = (kAlignK ? 0 : kLutK) + (kAlignV ? 0 : kLutV);
   // One ring slot holds one tile: K codes, V codes, K norms, V norms.
   static constexpr int kSlotK = kHasK ? kTile * NB * Fmt<KB>::kBlockBytes : 0;
   static constexpr int kSlotV = kHasV ? kTile * NB * Fmt<VB>::kBlockBytes : 0;
@@ -264,11 +314,15 @@ struct Smem {
   static constexpr int kSlotBytes = (kOffSlotVN + kSlotVN + 127) / 128 * 128;
   static constexpr int kWorkFloats = kCWarps * kMaxGroup * D;    // per-warp partials / qhat
   static constexpr int kResFloats = kMaxGroup * D;               // merged rotated-domain acc
-  static constexpr int kOffLutK = 0;
-  static constexpr int kOffLutV = kOffLutK + kLutK;
+  static constexpr int kOffLutK = 0;                       // dynamic, when not aligned
+  static constexpr int kOffLutV = kAlignK ? 0 : kLutK;
   static constexpr int kOffRing = (kDynLut + 127) / 128 * 128;
-  static constexpr int kOffWork = kOffRing + kCWarps * kDepth * kSlotBytes;
-  static constexpr int kOffRes = kOffWork + kWorkFloats * 4;
+  // The warp partials and the query scratch reuse the ring: the ring is empty
+  // (every copy waited for) whenever they are in use.
+  static constexpr int kRingBytes = kCWarps * kDepth * kSlotBytes;
+  static constexpr int kRingArea = kRingBytes > kWorkFloats * 4 ? kRingBytes : kWorkFloats * 4;
+  static constexpr int kOffWork = kOffRing;
+  static constexpr int kOffRes = kOffRing + kRingArea;
   static constexpr int kOffMisc = kOffRes + kResFloats * 4;
   // misc: warp m/l [kCWarps][8] x2, merged M/L/lse [8] x3, qexp [8], warp
   // totals [16], flags [4], reduction scratch [kCThreads] x2, merge factors.
@@ -355,17 +409,23 @@ __device__ __forceinline__ Segment locate(long long x, long long hi, const int* 
 // --------------------------------------------------------------- the kernel --
 
 template <int KB, int VB, int NB, int MODE>
-__global__ void __launch_bounds__(kThreads, TQ_DECODE_MIN_CTAS)
+__global__ void __launch_bounds__(kThreads, NB == 1 ? TQ_DECODE_MIN_CTAS : 2)
 decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   using SM = Smem<KB, VB, NB, MODE>;
   constexpr int D = SM::D;
   constexpr bool HASK = SM::kHasK, HASV = SM::kHasV;
   constexpr int KBB = Fmt<KB>::kBlockBytes, VBB = Fmt<VB>::kBlockBytes;
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(128) uint8_t slut[SM::kStaticBytes];
-  uint8_t* lut_base = SM::kStaticLut ? slut : smem;
-  uint8_t* lutK = lut_base + SM::kOffLutK;
-  uint8_t* lutV = lut_base + SM::kOffLutV;
+  __shared__ __align__(128) uint8_t rawLut[SM::kRawLut];
+  // shared-window addresses of the two tables
+  uint32_t lutK_s, lutV_s;
+  {
+    const uint32_t a = SM::kAMax ? (uint32_t)SM::kAMax : 16u;
+    const uint32_t first = (smem_addr(rawLut) + a - 1) & ~(a - 1);
+    const uint32_t second = first + (uint32_t)(SM::kKFirst ? SM::kAK : SM::kAV);
+    lutK_s = SM::kAlignK ? (SM::kKFirst ? first : second) : smem_addr(smem + SM::kOffLutK);
+    lutV_s = SM::kAlignV ? (SM::kKFirst ? second : first) : smem_addr(smem + SM::kOffLutV);
+  }
   uint8_t* ring = smem + SM::kOffRing;
   float* work = reinterpret_cast<float*>(smem + SM::kOffWork);
   float* res = reinterpret_cast<float*>(smem + SM::kOffRes);
@@ -386,6 +446,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = lane >> 2, g = lane & 3;
   const uint32_t lane4 = (uint32_t)lane * 4u;
+  const uint32_t lbK = lutK_s + lane4, lbV = lutV_s + lane4;
   const int G = p.q_heads / p.kv_heads;
   const int n_hg = (G + kMaxGroup - 1) / kMaxGroup;
   const int UB = p.kv_heads * n_hg;  // units per batch entry
@@ -395,14 +456,14 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     for (int e = tid; e < Fmt<KB>::kEntries * 32; e += kThreads) {
       const int ent = e >> 5;
       const float lo = p.kcent[ent & ((1 << KB) - 1)], hi = p.kcent[ent >> KB];
-      reinterpret_cast<uint32_t*>(lutK)[e] = pack_half2(lo, hi);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(lutK_s + 4u * e), "r"(pack_half2(lo, hi)) : "memory");
     }
   }
   if constexpr (HASV) {
     for (int e = tid; e < Fmt<VB>::kEntries * 32; e += kThreads) {
       const int ent = e >> 5;
       const float lo = p.vcent[ent & ((1 << VB) - 1)], hi = p.vcent[ent >> VB];
-      reinterpret_cast<uint32_t*>(lutV)[e] = pack_half2(lo, hi);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(lutV_s + 4u * e), "r"(pack_half2(lo, hi)) : "memory");
     }
   }
 
@@ -549,14 +610,12 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.0f, 0.0f};
 
-    auto compute = [&](const TileRegs<KB, VB, NB>& tr, int tile) {
-      const int t0 = tile * kTile;
-      // rows R and R+8 of the score tile are tokens 2R and 2R+1
-      const bool okR = t0 + 2 * R < len, okR8 = t0 + 2 * R + 1 < len;
-      float pR[2], pR8[2];
+    // Phase 1 of a tile: raw Hadamard-domain score sums per block (D2/D3),
+    // straight from the codes, in two independent accumulator chains.
+    struct Raw { float c[NB][4]; };
+    auto scores = [&](const TileRegs<KB, VB, NB>& tr) {
+      Raw r;
       if constexpr (HASK) {
-        // D2/D3: scores in the Hadamard domain, straight from the codes; two
-        // independent accumulator chains (even / odd k-steps)
         float ca[NB][4], cb[NB][4];
 #pragma unroll
         for (int blk = 0; blk < NB; ++blk) {
@@ -564,13 +623,28 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           for (int e = 0; e < 4; ++e) ca[blk][e] = cb[blk][e] = 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const uint32_t a0 = lds(lutK, lut_off(tr.k[0][blk], 2 * KB * (2 * j), 2 * KB, lane4));
-            const uint32_t a1 = lds(lutK, lut_off(tr.k[1][blk], 2 * KB * (2 * j), 2 * KB, lane4));
-            const uint32_t a2 = lds(lutK, lut_off(tr.k[0][blk], 2 * KB * (2 * j + 1), 2 * KB, lane4));
-            const uint32_t a3 = lds(lutK, lut_off(tr.k[1][blk], 2 * KB * (2 * j + 1), 2 * KB, lane4));
+            const uint32_t a0 = lut_get<SM::kAlignK>(tr.k[0][blk], 2 * KB * (2 * j), 2 * KB, lbK);
+            const uint32_t a1 = lut_get<SM::kAlignK>(tr.k[1][blk], 2 * KB * (2 * j), 2 * KB, lbK);
+            const uint32_t a2 = lut_get<SM::kAlignK>(tr.k[0][blk], 2 * KB * (2 * j + 1), 2 * KB, lbK);
+            const uint32_t a3 = lut_get<SM::kAlignK>(tr.k[1][blk], 2 * KB * (2 * j + 1), 2 * KB, lbK);
             mma16816((j & 1) ? cb[blk] : ca[blk], a0, a1, a2, a3, qf[blk][j][0], qf[blk][j][1]);
           }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) r.c[blk][e] = ca[blk][e] + cb[blk][e];
         }
+      }
+      return r;
+    };
+
+    // Phase 2 of a tile: scale and mask the scores, online softmax (D4) or the
+    // sparse-V gate (D5), then the V sum in the rotated domain (D6).
+    auto finish = [&](const TileRegs<KB, VB, NB>& tr, int tile, const Raw& raw, auto full_tag) {
+      constexpr bool FULL = decltype(full_tag)::value;
+      const int t0 = tile * kTile;
+      // rows R and R+8 of the score tile are tokens 2R and 2R+1
+      const bool okR = FULL || t0 + 2 * R < len, okR8 = FULL || t0 + 2 * R + 1 < len;
+      float pR[2], pR8[2];
+      if constexpr (HASK) {
         float sR[2], sR8[2];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -578,8 +652,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 #pragma unroll
           for (int blk = 0; blk < NB; ++blk) {
             const float2 kn = norm_pair<NB>(tr.kn, blk);
-            a = fmaf(ca[blk][cc] + cb[blk][cc], kn.x, a);
-            bb = fmaf(ca[blk][2 + cc] + cb[blk][2 + cc], kn.y, bb);
+            a = fmaf(raw.c[blk][cc], kn.x, a);
+            bb = fmaf(raw.c[blk][2 + cc], kn.y, bb);
           }
           sR[cc] = okR ? a * qmul[cc] : -INFINITY;
           sR8[cc] = okR8 ? bb * qmul[cc] : -INFINITY;
@@ -669,10 +743,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             const uint32_t b1 = movtrans(pack_half2(pR8[0] * sv1, pR8[1] * sv1));
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
-              const uint32_t x0 = lds(lutV, lut_off(tr.v[0][blk], 2 * VB * mt, 2 * VB, lane4));
-              const uint32_t x1 = lds(lutV, lut_off(tr.v[1][blk], 2 * VB * mt, 2 * VB, lane4));
-              const uint32_t x2 = lds(lutV, lut_off(tr.v[2][blk], 2 * VB * mt, 2 * VB, lane4));
-              const uint32_t x3 = lds(lutV, lut_off(tr.v[3][blk], 2 * VB * mt, 2 * VB, lane4));
+              const uint32_t x0 = lut_get<SM::kAlignV>(tr.v[0][blk], 2 * VB * mt, 2 * VB, lbV);
+              const uint32_t x1 = lut_get<SM::kAlignV>(tr.v[1][blk], 2 * VB * mt, 2 * VB, lbV);
+              const uint32_t x2 = lut_get<SM::kAlignV>(tr.v[2][blk], 2 * VB * mt, 2 * VB, lbV);
+              const uint32_t x3 = lut_get<SM::kAlignV>(tr.v[3][blk], 2 * VB * mt, 2 * VB, lbV);
               mma16816(acc[blk][mt], prmt(x0, x1, 0x5410), prmt(x0, x1, 0x7632),
                        prmt(x2, x3, 0x5410), prmt(x2, x3, 0x7632), b0, b1);
             }
@@ -687,6 +761,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       auto issue = [&](int tile, int slot) {
         const int t0 = tile * kTile;
         const int nval = min(kTile, len - t0);  // >= 1
+        const bool full = nval == kTile;
         const uint32_t sb = wring_s + (uint32_t)(slot * SM::kSlotBytes);
         if constexpr (HASK) {
           constexpr int kChunks = kTile * NB * KB;  // 16-byte chunks (KBB = 16 * KB)
@@ -696,13 +771,13 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           for (int c0 = 0; c0 < kChunks; c0 += 32) {
             const int c = c0 + lane;
             if (c < kChunks) {
-              const bool ok = c / kPerTok < nval;
+              const bool ok = full || c / kPerTok < nval;
               cp_async16(sb + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
             }
           }
           if (lane < 8 * NB) {  // norms: 4-byte pieces of the tile's 16*NB halves
             const int e = 2 * lane;  // first half of the piece
-            const int valid = max(0, min(2, nval * NB - e));
+            const int valid = full ? 2 : max(0, min(2, nval * NB - e));
             cp_async4(sb + SM::kOffSlotKN + 4u * lane, knp + (size_t)t0 * NB + (valid ? e : 0),
                       2u * (uint32_t)valid);
           }
@@ -715,13 +790,13 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           for (int c0 = 0; c0 < kChunks; c0 += 32) {
             const int c = c0 + lane;
             if (c < kChunks) {
-              const bool ok = c / kPerTok < nval;
+              const bool ok = full || c / kPerTok < nval;
               cp_async16(sb + SM::kOffSlotV + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
             }
           }
           if (lane < 8 * NB) {
             const int e = 2 * lane;
-            const int valid = max(0, min(2, nval * NB - e));
+            const int valid = full ? 2 : max(0, min(2, nval * NB - e));
             cp_async4(sb + SM::kOffSlotVN + 4u * lane, vnp + (size_t)t0 * NB + (valid ? e : 0),
                       2u * (uint32_t)valid);
           }
@@ -737,31 +812,37 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       const int first = seg_lo + cw;
       const int n_mine = first < seg_hi ? (seg_hi - first + kCWarps - 1) / kCWarps : 0;
 #pragma unroll
-      for (int i = 0; i < kDepth - 1; ++i) {
+      for (int i = 0; i < kDepth; ++i) {
         if (i < n_mine) issue(first + i * kCWarps, i);
         cp_async_commit();
       }
+      // Tile i of the warp sits in slot i % kDepth.  Once both halves of a
+      // tile are in registers, its slot is handed to tile i + kDepth, so the
+      // copy runs under the tile's arithmetic.
       for (int i = 0; i < n_mine; ++i) {
-        const int tile = first + i * kCWarps;
-        const int slot = i % kDepth;
-        cp_async_wait<kDepth - 2>();  // this warp's copies of tile i have landed
-        __syncwarp();
         TileRegs<KB, VB, NB> tr;
-        const uint8_t* sl = wring + (size_t)slot * SM::kSlotBytes;
+        const uint32_t sl = wring_s + (uint32_t)((i % kDepth) * SM::kSlotBytes);
+        cp_async_wait<kDepth - 1>();  // tile i has landed
+        __syncwarp();
         read_tile<KB, VB, NB, HASK, HASV>(tr, sl + koff, sl + voff, R);
         if constexpr (HASK) read_norms<NB>(tr.kn, sl + SM::kOffSlotKN, R);
         if constexpr (HASV) read_norms<NB>(tr.vn, sl + SM::kOffSlotVN, R);
-        compute(tr, tile);
-        // refill: tile i + kDepth - 1 goes to the slot freed by tile i - 1
-        __syncwarp();
-        if (i + kDepth - 1 < n_mine) issue(first + (i + kDepth - 1) * kCWarps, (i + kDepth - 1) % kDepth);
+        __syncwarp();  // no lane reads the slot any more
+        if (i + kDepth < n_mine) issue(first + (i + kDepth) * kCWarps, i % kDepth);
         cp_async_commit();
+        const int tile = first + i * kCWarps;
+        const Raw raw = scores(tr);
+        if (tile * kTile + kTile <= len)
+          finish(tr, tile, raw, std::true_type{});
+        else
+          finish(tr, tile, raw, std::false_type{});
       }
       cp_async_wait<0>();
       __syncwarp();
     }
 
     // ---- warp partials to shared memory -----------------------------------
+    consumer_sync();  // every warp is done with its ring, which holds the partials
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
       float l = l_run[cc];
