@@ -50,15 +50,18 @@ namespace {
 #ifndef TQ_DECODE_MIN_CTAS
 #define TQ_DECODE_MIN_CTAS 3
 #endif
+#ifndef TQ_KCHAINS
+#define TQ_KCHAINS 2  // independent accumulator chains of the score MMAs
+#endif
 #ifndef TQ_RING_DEPTH
 #define TQ_RING_DEPTH 4
 #endif
+constexpr int kKChains = TQ_KCHAINS;
 constexpr int kCWarps = TQ_DECODE_WARPS;        // warps per CTA
 constexpr int kCThreads = 32 * kCWarps;
 constexpr int kThreads = kCThreads;
-constexpr int kDepth = TQ_RING_DEPTH;           // tiles per warp ring (in flight: kDepth - 1)
+constexpr int kDepth = TQ_RING_DEPTH;           // tiles per warp ring (all in flight)
 constexpr float kTau = 6.0f;                    // lazy-rescale threshold (log2 units)
-constexpr int kStaticLutLimit = 40 * 1024;      // tables up to this size are static shared
 constexpr int kMergeChunk = 64;                 // partials merged per pass of the final merge
 
 enum Mode { kFused = 0, kScores = 1, kSparseV = 2 };
@@ -301,7 +304,6 @@ struct Smem {
   static constexpr int kAMax = kAK > kAV ? kAK : kAV;
   static constexpr int kRawLut = (kAK + kAV) ? kAK + kAV + kAMax : 16;
   static constexpr bool kKFirst = kAK >= kAV;
-  static constexpr bool kStaticLut = false;  // unaligned tables, if any, are dynamic
   static constexpr int kDynLut = (kAlignK ? 0 : kLutK) + (kAlignV ? 0 : kLutV);
   // One ring slot holds one tile: K codes, V codes, K norms, V norms.
   static constexpr int kSlotK = kHasK ? kTile * NB * Fmt<KB>::kBlockBytes : 0;
@@ -327,27 +329,45 @@ struct Smem {
   // misc: warp m/l [kCWarps][8] x2, merged M/L/lse [8] x3, qexp [8], warp
   // totals [16], flags [4], reduction scratch [kCThreads] x2, merge factors.
   static constexpr int kMiscFloats = 2 * kCWarps * kMaxGroup + 4 * kMaxGroup + 16 + 4 +
-                                     2 * kCThreads + kMergeChunk * kMaxGroup;
+                                     2 * kCThreads + 2 * kMergeChunk * kMaxGroup;
   static constexpr int kOffPrefix = kOffMisc + kMiscFloats * 4;
   static size_t bytes(int batch) { return (size_t)kOffPrefix + (size_t)(batch + 1) * 4; }
 };
 
-// Per-head (M, L) = (max m, sum l * 2^(m - M)) over the partials of one unit,
-// using every consumer thread: thread t takes head t % 8 and every
-// (kCThreads/8)-th partial, folding them in a fixed order; the running pairs
-// of a head are then combined in a fixed order.  Partials of CTAs whose range
-// is empty are skipped.
+// (m, l) of partials c0 .. c0+n-1 of one unit into shared memory, every load
+// in flight at once; heads >= Gu and CTAs whose range is empty get (-inf, 0).
+__device__ __forceinline__ void stage_ml(const float* slot_ml, long long c0, int n, long long parts,
+                                         long long T, long long unit, int Gu, float* sm, float* sl) {
+  for (int i = threadIdx.x; i < n * kMaxGroup; i += kCThreads) {
+    const long long c = c0 + i / kMaxGroup;
+    const int hd = i % kMaxGroup;
+    float2 ml = make_float2(-INFINITY, 0.0f);
+    if (hd < Gu && c * T / parts != (c + 1) * T / parts)
+      ml = __ldcg(reinterpret_cast<const float2*>(slot_ml + ((c + unit) * kMaxGroup + hd) * 2));
+    sm[i] = ml.x;
+    sl[i] = ml.y;
+  }
+}
+
+// Per-head (M, L) = (max m, sum l * 2^(m - M)) over the partials c_first ..
+// c_last of one unit.  Partials are staged kMergeChunk at a time; thread t
+// folds head t % 8 of every (kCThreads/8)-th staged partial, then the running
+// pairs of a head are combined, all in a fixed order.  On return sm/sl hold
+// the last staged chunk.
 __device__ __forceinline__ void unit_stats(const float* slot_ml, long long c_first, long long c_last,
                                            long long parts, long long T, long long unit, int Gu,
-                                           float* red_m, float* red_l, float* outM, float* outL) {
+                                           float* sm, float* sl, float* red_m, float* red_l,
+                                           float* outM, float* outL) {
   constexpr int J = kCThreads / kMaxGroup;
   const int tid = threadIdx.x, hd = tid % kMaxGroup, j = tid / kMaxGroup;
   float m = -INFINITY, l = 0.0f;
-  if (hd < Gu) {
-    for (long long c = c_first + j; c <= c_last; c += J) {
-      if (c * T / parts == (c + 1) * T / parts) continue;
-      const float* ml = slot_ml + ((c + unit) * kMaxGroup + hd) * 2;
-      const float mc = __ldcg(ml), lc = __ldcg(ml + 1);
+  for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
+    const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
+    consumer_sync();  // the previous chunk has been folded
+    stage_ml(slot_ml, c0, n, parts, T, unit, Gu, sm, sl);
+    consumer_sync();
+    for (int k = j; k < n; k += J) {
+      const float mc = sm[k * kMaxGroup + hd], lc = sl[k * kMaxGroup + hd];
       if (mc == -INFINITY) continue;
       if (mc > m) {
         l = l * ex2(m - mc) + lc;
@@ -408,13 +428,20 @@ __device__ __forceinline__ Segment locate(long long x, long long hi, const int* 
 
 // --------------------------------------------------------------- the kernel --
 
-template <int KB, int VB, int NB, int MODE>
+template <int KB, int VB, int NB, int MODE, int GQ>
 __global__ void __launch_bounds__(kThreads, NB == 1 ? TQ_DECODE_MIN_CTAS : 2)
 decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   using SM = Smem<KB, VB, NB, MODE>;
   constexpr int D = SM::D;
   constexpr bool HASK = SM::kHasK, HASV = SM::kHasV;
   constexpr int KBB = Fmt<KB>::kBlockBytes, VBB = Fmt<VB>::kBlockBytes;
+  // GQ == 4 (at most four query heads per unit): score columns 4..7 repeat
+  // heads 0..3, and the V products use the eight MMA columns as (head, dim
+  // parity) pairs, so V fragments come straight from the table.  GQ == 8:
+  // one column per head, V fragments re-paired by token.
+  static_assert(GQ == 4 || GQ == 8, "GQ");
+  constexpr bool kDup = GQ == 4;
+  constexpr int kMT = kDup ? 4 : 8;  // V accumulator tiles per 128-block
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(128) uint8_t rawLut[SM::kRawLut];
   // shared-window addresses of the two tables
@@ -440,13 +467,17 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   int* flag = wtot + 16;                              // [4]
   float* red_m = reinterpret_cast<float*>(flag + 4);  // [kCThreads]
   float* red_l = red_m + kCThreads;                   // [kCThreads]
-  float* fac = red_l + kCThreads;                     // [kMergeChunk][8]
+  float* fac = red_l + kCThreads;                     // [kMergeChunk][8] staged m, then weights
+  float* stl = fac + kMergeChunk * kMaxGroup;         // [kMergeChunk][8] staged l
   int* prefix = reinterpret_cast<int*>(smem + SM::kOffPrefix);  // [B+1] tiles per batch, prefix
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int R = lane >> 2, g = lane & 3;
   const uint32_t lane4 = (uint32_t)lane * 4u;
   const uint32_t lbK = lutK_s + lane4, lbV = lutV_s + lane4;
+  // kDup B fragments: a token's weight in the low half (s' = 0, R < 4) or
+  // the high half (s' = 1) of the register, zero in the other
+  const uint32_t selLo = R < 4 ? 0x4410u : 0x1044u, selHi = R < 4 ? 0x4432u : 0x3244u;
   const int G = p.q_heads / p.kv_heads;
   const int n_hg = (G + kMaxGroup - 1) / kMaxGroup;
   const int UB = p.kv_heads * n_hg;  // units per batch entry
@@ -538,7 +569,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     float lse2[2] = {0.0f, 0.0f};
     if constexpr (HASK) {
       float* qs = work;  // [8][D]
-      for (int i = tid; i < kMaxGroup * D; i += kCThreads) {
+      constexpr int kQRows = kDup ? 4 : kMaxGroup;
+      for (int i = tid; i < kQRows * D; i += kCThreads) {
         const int j = i / D, d = i % D;
         float v = 0.0f;
         if (j < Gu) {
@@ -552,7 +584,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       }
       consumer_sync();
       for (int s = 1; s < kBlock; s <<= 1) {
-        for (int i = tid; i < kMaxGroup * D / 2; i += kCThreads) {
+        for (int i = tid; i < kQRows * D / 2; i += kCThreads) {
           const int j = i / (D / 2), rem = i % (D / 2);
           const int a = (rem / s) * 2 * s + (rem % s);
           float* row = qs + j * D;
@@ -564,7 +596,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       }
       // power-of-two scale per head so fp16 fragments neither overflow nor
       // fall into subnormals
-      for (int j = cw; j < kMaxGroup; j += kCWarps) {
+      for (int j = cw; j < kQRows; j += kCWarps) {
         float mx = 0.0f;
         for (int d = lane; d < D; d += 32) mx = fmaxf(mx, fabsf(qs[j * D + d]));
 #pragma unroll
@@ -572,65 +604,73 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         if (lane == 0) qexp[j] = (mx > 0.0f) ? (ilogbf(mx) - 13) : 0;
       }
       consumer_sync();
-      const float qsc = ldexpf(1.0f, -qexp[R]);
+      const float qsc = ldexpf(1.0f, -qexp[kDup ? (R & 3) : R]);
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float* q4 = qs + R * D + blk * kBlock + 32 * g + 4 * j;
+          const float* q4 = qs + (kDup ? (R & 3) : R) * D + blk * kBlock + 32 * g + 4 * j;
           qf[blk][j][0] = pack_half2(q4[0] * qsc, q4[1] * qsc);
           qf[blk][j][1] = pack_half2(q4[2] * qsc, q4[3] * qsc);
         }
       }
-      qmul[0] = p.score_mult * ldexpf(1.0f, qexp[2 * g]);
-      qmul[1] = p.score_mult * ldexpf(1.0f, qexp[2 * g + 1]);
+      qmul[0] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g) & 3 : 2 * g]);
+      qmul[1] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g + 1) & 3 : 2 * g + 1]);
       consumer_sync();  // work area is reused below
     }
     if constexpr (MODE == kSparseV) {
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote
       const long long P1 = p1_ctas;
-      unit_stats(p.slot_ml, cta_of(Su, P1), cta_of(Su + nt - 1, P1), P1, T, unit, Gu, red_m, red_l,
+      unit_stats(p.slot_ml, cta_of(Su, P1), cta_of(Su + nt - 1, P1), P1, T, unit, Gu, fac, stl, red_m, red_l,
                  u_M, u_L);
       if (tid < Gu) u_lse[tid] = u_M[tid] + __log2f(u_L[tid]);
       consumer_sync();
-      lse2[0] = (2 * g < Gu) ? u_lse[2 * g] : 0.0f;
-      lse2[1] = (2 * g + 1 < Gu) ? u_lse[2 * g + 1] : 0.0f;
+      const int hd0 = kDup ? (2 * g) & 3 : 2 * g, hd1 = kDup ? (2 * g + 1) & 3 : 2 * g + 1;
+      lse2[0] = (hd0 < Gu) ? u_lse[hd0] : 0.0f;
+      lse2[1] = (hd1 < Gu) ? u_lse[hd1] : 0.0f;
     }
     const float log2_thr = (MODE == kSparseV) ? __log2f(p.sparse_thr) : 0.0f;
 
     // ---- warp loop over this segment's stages -----------------------------
-    float acc[NB][8][4];
+    float acc[NB][kMT][4];
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
+      for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[blk][mt][e] = 0.0f;
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.0f, 0.0f};
 
     // Phase 1 of a tile: raw Hadamard-domain score sums per block (D2/D3),
-    // straight from the codes, in two independent accumulator chains.
+    // straight from the codes, in kKChains independent accumulator chains.
     struct Raw { float c[NB][4]; };
     auto scores = [&](const TileRegs<KB, VB, NB>& tr) {
-      Raw r;
+      Raw r{};
       if constexpr (HASK) {
-        float ca[NB][4], cb[NB][4];
+        float ca[kKChains][NB][4];
 #pragma unroll
         for (int blk = 0; blk < NB; ++blk) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) ca[blk][e] = cb[blk][e] = 0.0f;
+          for (int c = 0; c < kKChains; ++c)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ca[c][blk][e] = 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint32_t a0 = lut_get<SM::kAlignK>(tr.k[0][blk], 2 * KB * (2 * j), 2 * KB, lbK);
             const uint32_t a1 = lut_get<SM::kAlignK>(tr.k[1][blk], 2 * KB * (2 * j), 2 * KB, lbK);
             const uint32_t a2 = lut_get<SM::kAlignK>(tr.k[0][blk], 2 * KB * (2 * j + 1), 2 * KB, lbK);
             const uint32_t a3 = lut_get<SM::kAlignK>(tr.k[1][blk], 2 * KB * (2 * j + 1), 2 * KB, lbK);
-            mma16816((j & 1) ? cb[blk] : ca[blk], a0, a1, a2, a3, qf[blk][j][0], qf[blk][j][1]);
+            mma16816(ca[j % kKChains][blk], a0, a1, a2, a3, qf[blk][j][0], qf[blk][j][1]);
           }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) r.c[blk][e] = ca[blk][e] + cb[blk][e];
+          for (int e = 0; e < 4; ++e) {
+            float t = ca[0][blk][e];
+#pragma unroll
+            for (int c = 1; c < kKChains; ++c) t += ca[c][blk][e];
+            r.c[blk][e] = t;
+          }
         }
       }
       return r;
@@ -661,8 +701,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         if constexpr (MODE == kScores) {
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
-            const int hd = 2 * g + cc;
-            if (hd < Gu) {
+            const int hd = 2 * g + cc;  // columns 4..7 repeat heads 0..3 when kDup
+            if (hd < Gu && (!kDup || g < 2)) {
               float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap + t0 + 2 * R;
               if (okR8) {
                 *reinterpret_cast<float2*>(srow) = make_float2(sR[cc], sR8[cc]);
@@ -690,7 +730,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 #pragma unroll
                 for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
-                  for (int mt = 0; mt < 8; ++mt) {
+                  for (int mt = 0; mt < kMT; ++mt) {
                     acc[blk][mt][cc] *= alpha;
                     acc[blk][mt][2 + cc] *= alpha;
                   }
@@ -709,7 +749,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         // pass 2 of sparse-V: normalised weights from the stored scores (D5)
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          const int hd = 2 * g + cc;
+          const int hd = kDup ? (2 * g + cc) & 3 : 2 * g + cc;
           float wR = 0.0f, wR8 = 0.0f;
           if (hd < Gu) {
             const float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap + t0 + 2 * R;
@@ -739,16 +779,39 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           for (int blk = 0; blk < NB; ++blk) {
             const float2 vn = norm_pair<NB>(tr.vn, blk);
             const float sv0 = vn.x * (1.0f / kBlock), sv1 = vn.y * (1.0f / kBlock);
+            // P^T fragments: lane (R, g) gets tokens 4g, 4g+2 (b0) and
+            // 4g+1, 4g+3 (b1) of score column R
             const uint32_t b0 = movtrans(pack_half2(pR[0] * sv0, pR[1] * sv0));
             const uint32_t b1 = movtrans(pack_half2(pR8[0] * sv1, pR8[1] * sv1));
+            if constexpr (kDup) {
+              // k = 2*tau + s, column n = h + 4*s': the product pairs the
+              // weight of token tau with dim 2*pair + s only when s == s', so
+              // each A register is one token's pair of adjacent dims.  Rows R,
+              // R+8 of tile q are dim pairs 8R+2q, 8R+2q+1.
+              const uint32_t pa0 = prmt(b0, 0u, selLo), pa1 = prmt(b0, 0u, selHi);
+              const uint32_t pb0 = prmt(b1, 0u, selLo), pb1 = prmt(b1, 0u, selHi);
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-              const uint32_t x0 = lut_get<SM::kAlignV>(tr.v[0][blk], 2 * VB * mt, 2 * VB, lbV);
-              const uint32_t x1 = lut_get<SM::kAlignV>(tr.v[1][blk], 2 * VB * mt, 2 * VB, lbV);
-              const uint32_t x2 = lut_get<SM::kAlignV>(tr.v[2][blk], 2 * VB * mt, 2 * VB, lbV);
-              const uint32_t x3 = lut_get<SM::kAlignV>(tr.v[3][blk], 2 * VB * mt, 2 * VB, lbV);
-              mma16816(acc[blk][mt], prmt(x0, x1, 0x5410), prmt(x0, x1, 0x7632),
-                       prmt(x2, x3, 0x5410), prmt(x2, x3, 0x7632), b0, b1);
+              for (int q = 0; q < 4; ++q) {
+                const int f0 = 2 * VB * (2 * q), f1 = 2 * VB * (2 * q + 1);
+                mma16816(acc[blk][q], lut_get<SM::kAlignV>(tr.v[0][blk], f0, 2 * VB, lbV),
+                         lut_get<SM::kAlignV>(tr.v[0][blk], f1, 2 * VB, lbV),
+                         lut_get<SM::kAlignV>(tr.v[1][blk], f0, 2 * VB, lbV),
+                         lut_get<SM::kAlignV>(tr.v[1][blk], f1, 2 * VB, lbV), pa0, pa1);
+                mma16816(acc[blk][q], lut_get<SM::kAlignV>(tr.v[2][blk], f0, 2 * VB, lbV),
+                         lut_get<SM::kAlignV>(tr.v[2][blk], f1, 2 * VB, lbV),
+                         lut_get<SM::kAlignV>(tr.v[3][blk], f0, 2 * VB, lbV),
+                         lut_get<SM::kAlignV>(tr.v[3][blk], f1, 2 * VB, lbV), pb0, pb1);
+              }
+            } else {
+#pragma unroll
+              for (int mt = 0; mt < 8; ++mt) {
+                const uint32_t x0 = lut_get<SM::kAlignV>(tr.v[0][blk], 2 * VB * mt, 2 * VB, lbV);
+                const uint32_t x1 = lut_get<SM::kAlignV>(tr.v[1][blk], 2 * VB * mt, 2 * VB, lbV);
+                const uint32_t x2 = lut_get<SM::kAlignV>(tr.v[2][blk], 2 * VB * mt, 2 * VB, lbV);
+                const uint32_t x3 = lut_get<SM::kAlignV>(tr.v[3][blk], 2 * VB * mt, 2 * VB, lbV);
+                mma16816(acc[blk][mt], prmt(x0, x1, 0x5410), prmt(x0, x1, 0x7632),
+                         prmt(x2, x3, 0x5410), prmt(x2, x3, 0x7632), b0, b1);
+              }
             }
           }
         }
@@ -849,22 +912,37 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       l += __shfl_xor_sync(0xffffffffu, l, 4);
       l += __shfl_xor_sync(0xffffffffu, l, 8);
       l += __shfl_xor_sync(0xffffffffu, l, 16);
-      if (R == 0) {
+      if (R == 0 && (!kDup || g < 2)) {
         w_m[cw * kMaxGroup + 2 * g + cc] = m_run[cc];
         w_l[cw * kMaxGroup + 2 * g + cc] = l;
       }
     }
     if constexpr (HASV) {
+      if constexpr (kDup) {
+        // element e of tile q: column 2g + (e & 1) = head h + 4 s' (s' = g >> 1),
+        // row R + 8 (e >> 1) = dim pair 8R + 2q + (e >> 1), dim 2 pair + s'
 #pragma unroll
-      for (int blk = 0; blk < NB; ++blk)
+        for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          const int d0 = blk * kBlock + 16 * R + 2 * mt;
-          float* w0 = work + (cw * kMaxGroup + 2 * g) * D + d0;
-          float* w1 = work + (cw * kMaxGroup + 2 * g + 1) * D + d0;
-          *reinterpret_cast<float2*>(w0) = make_float2(acc[blk][mt][0], acc[blk][mt][2]);
-          *reinterpret_cast<float2*>(w1) = make_float2(acc[blk][mt][1], acc[blk][mt][3]);
-        }
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int h = (2 * g + (e & 1)) & 3;
+              const int d = blk * kBlock + 16 * R + 4 * q + 2 * (e >> 1) + (g >> 1);
+              work[(cw * kMaxGroup + h) * D + d] = acc[blk][q][e];
+            }
+      } else {
+#pragma unroll
+        for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            const int d0 = blk * kBlock + 16 * R + 2 * mt;
+            float* w0 = work + (cw * kMaxGroup + 2 * g) * D + d0;
+            float* w1 = work + (cw * kMaxGroup + 2 * g + 1) * D + d0;
+            *reinterpret_cast<float2*>(w0) = make_float2(acc[blk][mt][0], acc[blk][mt][2]);
+            *reinterpret_cast<float2*>(w1) = make_float2(acc[blk][mt][1], acc[blk][mt][3]);
+          }
+      }
     }
     consumer_sync();
 
@@ -934,39 +1012,54 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         if (finalize) {
           __threadfence();
           const long long c_first = cta_of(Su, P), c_last = cta_of(Su + nt - 1, P);
-          if constexpr (HASK) unit_stats(p.slot_ml, c_first, c_last, P, T, unit, Gu, red_m, red_l, u_M, u_L);
+          if constexpr (HASK)
+            unit_stats(p.slot_ml, c_first, c_last, P, T, unit, Gu, fac, stl, red_m, red_l, u_M, u_L);
           for (int i = tid; i < Gu * D; i += kCThreads) res[i] = 0.0f;
+          const bool one_chunk = c_last - c_first < kMergeChunk;
           for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
-            // weights 2^(m_c - M) of this chunk's partials (0 for empty ranges)
-            for (int i = tid; i < kMergeChunk * kMaxGroup; i += kCThreads) {
-              const long long c = c0 + i / kMaxGroup;
-              const int hd = i % kMaxGroup;
-              float f = 0.0f;
-              if (c <= c_last && hd < Gu && c * T / P != (c + 1) * T / P) {
-                f = 1.0f;
-                if constexpr (HASK) {
-                  const float mc = __ldcg(p.slot_ml + ((c + unit) * kMaxGroup + hd) * 2);
-                  f = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[hd]);
-                }
+            const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
+            // weights 2^(m_c - M) of this chunk's partials (0 for empty ranges;
+            // without scores, 1 for every non-empty range)
+            if constexpr (HASK) {
+              if (!one_chunk) {  // else unit_stats left this chunk staged
+                consumer_sync();
+                stage_ml(p.slot_ml, c0, n, P, T, unit, Gu, fac, stl);
+                consumer_sync();
               }
-              fac[i] = f;
+              for (int i = tid; i < n * kMaxGroup; i += kCThreads) {
+                const float mc = fac[i];
+                fac[i] = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[i % kMaxGroup]);
+              }
+            } else {
+              consumer_sync();
+              for (int i = tid; i < n * kMaxGroup; i += kCThreads) {
+                const long long c = c0 + i / kMaxGroup;
+                fac[i] = (i % kMaxGroup < Gu && c * T / P != (c + 1) * T / P) ? 1.0f : 0.0f;
+              }
             }
             consumer_sync();
-            const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
-            for (int i = tid; i < Gu * D; i += kCThreads) {
-              const int hd = i / D, d = i % D;
-              const float* src = p.slot_acc + ((c0 + unit) * kMaxGroup + hd) * D + d;
-              float sacc = res[i];
-#pragma unroll 8
+            // four consecutive dims per thread, many partials in flight (the
+            // merge is on the critical path of the whole launch)
+            for (int i = tid; i < Gu * D / 4; i += kCThreads) {
+              const int hd = (4 * i) / D, d = (4 * i) % D;
+              const float4* src =
+                  reinterpret_cast<const float4*>(p.slot_acc + ((c0 + unit) * kMaxGroup + hd) * D + d);
+              float4 sacc = reinterpret_cast<const float4*>(res)[i];
+#pragma unroll 16
               for (int cc = 0; cc < n; ++cc) {
                 const float f = fac[cc * kMaxGroup + hd];
-                const float a = __ldcg(src + (size_t)cc * kMaxGroup * D);
-                sacc = (f != 0.0f) ? fmaf(a, f, sacc) : sacc;
+                const float4 a = __ldcg(src + (size_t)cc * kMaxGroup * D / 4);
+                if (f != 0.0f) {  // a partial that was never written may hold anything
+                  sacc.x = fmaf(a.x, f, sacc.x);
+                  sacc.y = fmaf(a.y, f, sacc.y);
+                  sacc.z = fmaf(a.z, f, sacc.z);
+                  sacc.w = fmaf(a.w, f, sacc.w);
+                }
               }
-              res[i] = sacc;
+              reinterpret_cast<float4*>(res)[i] = sacc;
             }
-            consumer_sync();
           }
+          consumer_sync();
           if (tid == 0) p.tickets[unit] = 0u;
           consumer_sync();
         }
@@ -1002,11 +1095,11 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 
 // --------------------------------------------------------------- launching --
 
-template <int KB, int VB, int NB, int MODE>
+template <int KB, int VB, int NB, int MODE, int GQ>
 int run(const DecodeParams& p, cudaStream_t stream, int p1_ctas, int* ctas_out) {
   using SM = Smem<KB, VB, NB, MODE>;
   const size_t smem = SM::bytes(p.batch);
-  auto kern = decode_kernel<KB, VB, NB, MODE>;
+  auto kern = decode_kernel<KB, VB, NB, MODE, GQ>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
   static int cached_sms[64] = {0};
@@ -1032,22 +1125,28 @@ int run(const DecodeParams& p, cudaStream_t stream, int p1_ctas, int* ctas_out) 
   return TQ_OK;
 }
 
-template <int KB, int VB, int NB>
+template <int KB, int VB, int NB, int GQ>
 int dispatch_modes(const DecodeParams& p, cudaStream_t stream) {
   if (p.sparse_thr > 0.0f) {
     int p1 = 0;
-    int st = run<KB, 2, NB, kScores>(p, stream, 0, &p1);
+    int st = run<KB, 2, NB, kScores, GQ>(p, stream, 0, &p1);
     if (st != TQ_OK) return st;
-    return run<2, VB, NB, kSparseV>(p, stream, p1, nullptr);
+    return run<2, VB, NB, kSparseV, GQ>(p, stream, p1, nullptr);
   }
-  return run<KB, VB, NB, kFused>(p, stream, 0, nullptr);
+  return run<KB, VB, NB, kFused, GQ>(p, stream, 0, nullptr);
+}
+
+template <int KB, int VB, int NB>
+int dispatch_gq(const DecodeParams& p, cudaStream_t stream) {
+  if (p.q_heads / p.kv_heads <= 4) return dispatch_modes<KB, VB, NB, 4>(p, stream);
+  return dispatch_modes<KB, VB, NB, 8>(p, stream);
 }
 
 template <int KB, int VB>
 int dispatch_nb(const DecodeParams& p, cudaStream_t stream) {
   switch (p.head_dim / kBlock) {
-    case 1: return dispatch_modes<KB, VB, 1>(p, stream);
-    case 2: return dispatch_modes<KB, VB, 2>(p, stream);
+    case 1: return dispatch_gq<KB, VB, 1>(p, stream);
+    case 2: return dispatch_gq<KB, VB, 2>(p, stream);
   }
   return TQ_ERR_UNSUPPORTED;
 }
