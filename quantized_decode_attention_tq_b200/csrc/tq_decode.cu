@@ -45,13 +45,19 @@ namespace tq {
 namespace {
 
 #ifndef TQ_DECODE_WARPS
-#define TQ_DECODE_WARPS 4
+#define TQ_DECODE_WARPS 16
 #endif
 #ifndef TQ_DECODE_MIN_CTAS
-#define TQ_DECODE_MIN_CTAS 3
+#define TQ_DECODE_MIN_CTAS 1
+#endif
+#ifndef TQ_DECODE_MIN_CTAS_WIDE  // head_dim 256 kernels
+#define TQ_DECODE_MIN_CTAS_WIDE (TQ_DECODE_MIN_CTAS > 2 ? 2 : TQ_DECODE_MIN_CTAS)
 #endif
 #ifndef TQ_KCHAINS
 #define TQ_KCHAINS 2  // independent accumulator chains of the score MMAs
+#endif
+#ifndef TQ_SWITCH_TILES
+#define TQ_SWITCH_TILES 96  // cost of starting another unit inside a CTA, in tiles
 #endif
 #ifndef TQ_RING_DEPTH
 #define TQ_RING_DEPTH 4
@@ -60,7 +66,8 @@ constexpr int kKChains = TQ_KCHAINS;
 constexpr int kCWarps = TQ_DECODE_WARPS;        // warps per CTA
 constexpr int kCThreads = 32 * kCWarps;
 constexpr int kThreads = kCThreads;
-constexpr int kDepth = TQ_RING_DEPTH;           // tiles per warp ring (all in flight)
+constexpr int kRingDepth = TQ_RING_DEPTH;       // tiles per warp ring (all in flight), at most
+constexpr int kMaxSmem = 227 * 1024;            // shared memory of one CTA (static + dynamic)
 constexpr float kTau = 6.0f;                    // lazy-rescale threshold (log2 units)
 constexpr int kMergeChunk = 64;                 // partials merged per pass of the final merge
 
@@ -319,6 +326,15 @@ struct Smem {
   static constexpr int kOffLutK = 0;                       // dynamic, when not aligned
   static constexpr int kOffLutV = kAlignK ? 0 : kLutK;
   static constexpr int kOffRing = (kDynLut + 127) / 128 * 128;
+  // misc: warp m/l [kCWarps][8] x2, merged M/L/lse [8] x3, qexp [8], warp
+  // totals [16], flags [4], reduction scratch [kCThreads] x2, merge factors.
+  static constexpr int kMiscFloats = 2 * kCWarps * kMaxGroup + 4 * kMaxGroup + 16 + 4 +
+                                     2 * kCThreads + 2 * kMergeChunk * kMaxGroup;
+  // Ring depth: kRingDepth tiles per warp when they fit next to everything
+  // else (the batch prefix counted at its largest), fewer otherwise.
+  static constexpr int kFixed = kRawLut + kOffRing + (kResFloats + kMiscFloats) * 4 + (kMaxBatch + 1) * 4;
+  static constexpr int kFit = (kMaxSmem - kFixed) / (kCWarps * kSlotBytes);
+  static constexpr int kDepth = kFit >= kRingDepth ? kRingDepth : (kFit < 1 ? 1 : kFit);
   // The warp partials and the query scratch reuse the ring: the ring is empty
   // (every copy waited for) whenever they are in use.
   static constexpr int kRingBytes = kCWarps * kDepth * kSlotBytes;
@@ -326,23 +342,105 @@ struct Smem {
   static constexpr int kOffWork = kOffRing;
   static constexpr int kOffRes = kOffRing + kRingArea;
   static constexpr int kOffMisc = kOffRes + kResFloats * 4;
-  // misc: warp m/l [kCWarps][8] x2, merged M/L/lse [8] x3, qexp [8], warp
-  // totals [16], flags [4], reduction scratch [kCThreads] x2, merge factors.
-  static constexpr int kMiscFloats = 2 * kCWarps * kMaxGroup + 4 * kMaxGroup + 16 + 4 +
-                                     2 * kCThreads + 2 * kMergeChunk * kMaxGroup;
   static constexpr int kOffPrefix = kOffMisc + kMiscFloats * 4;
   static size_t bytes(int batch) { return (size_t)kOffPrefix + (size_t)(batch + 1) * 4; }
 };
 
+// Unnormalised Walsh-Hadamard transform of each 128-block of one row held by
+// a warp: lane l holds elements 4l..4l+3 of every block.  Strides 1 and 2 are
+// in-lane, strides 4..64 pair lane l with lane l ^ (stride / 4); the lower
+// index of a pair gets u + w, the upper u - w.
+template <int NB>
+__device__ __forceinline__ void wht_rows(float (&v)[NB][4], int lane) {
+#pragma unroll
+  for (int blk = 0; blk < NB; ++blk) {
+    const float t0 = v[blk][0] + v[blk][1], t1 = v[blk][0] - v[blk][1];
+    const float t2 = v[blk][2] + v[blk][3], t3 = v[blk][2] - v[blk][3];
+    v[blk][0] = t0 + t2;
+    v[blk][2] = t0 - t2;
+    v[blk][1] = t1 + t3;
+    v[blk][3] = t1 - t3;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[blk][k], m);
+        v[blk][k] = (lane & m) ? o - v[blk][k] : v[blk][k] + o;
+      }
+    }
+  }
+}
+
+// How the flattened (unit, tile) space [0, T) is split over the persistent
+// CTAs.  Every unit's tiles cost 1 each and starting a unit costs kSwitchTiles
+// more (its query preparation, the drained copy ring, the partial's merge
+// and publication), so a CTA whose range spans two units gets fewer tiles:
+// CTA c takes the tiles whose cost falls in [c, c+1) * Ctot / P.  The cost
+// before batch entry b is UB * (prefix[b] + kSwitchTiles * b).  A cost that
+// falls between two units maps to the start of the second, so a cut there
+// adds no segment.  Results do not depend on the split (each part is computed
+// and merged in a fixed order); it only moves where the CTAs end.
+constexpr long long kSwitchTiles = TQ_SWITCH_TILES;
+
+// floor(a / b) for 0 <= a, 0 < b, both below 2^52: the double quotient is
+// within one of the exact one, and one integer step corrects it (a 64-bit
+// integer division is a long instruction sequence on the GPU).
+__device__ __forceinline__ long long fdiv(long long a, long long b) {
+  long long q = (long long)((double)a / (double)b);
+  if (q * b > a) --q; else if ((q + 1) * b <= a) ++q;
+  return q;
+}
+
+struct Split {
+  const int* prefix;  // [B+1] tiles per batch entry, exclusive prefix (shared memory)
+  int B, UB;
+  long long P, T, Ctot;
+  __device__ Split(const int* pre, int batch, int ub, long long parts)
+      : prefix(pre), B(batch), UB(ub), P(parts) {
+    T = (long long)pre[batch] * ub;
+    Ctot = (long long)ub * ((long long)pre[batch] + kSwitchTiles * batch);
+  }
+  // first tile of part c (c = P gives T)
+  __device__ long long start(long long c) const {
+    if (c >= P) return T;
+    const long long y = fdiv(c * Ctot, P);
+    int bl = 0, bh = B;  // largest b with cost(b) <= y
+    while (bh - bl > 1) {
+      const int mid = (bl + bh) >> 1;
+      if ((long long)UB * (prefix[mid] + kSwitchTiles * mid) <= y) bl = mid; else bh = mid;
+    }
+    const long long nt = prefix[bl + 1] - prefix[bl];
+    const long long rem = y - (long long)UB * (prefix[bl] + kSwitchTiles * bl);
+    const long long r = fdiv(rem, nt + kSwitchTiles), t = rem - r * (nt + kSwitchTiles);
+    return (long long)UB * prefix[bl] + r * nt + min(t, nt);
+  }
+  __device__ bool empty(long long c) const { return start(c) == start(c + 1); }
+  // The part whose range holds tile x (0 <= x < T): the last c whose cost
+  // floor(c * Ctot / P) is at most x's cost F.
+  __device__ long long part_of(long long x) const {
+    int bl = 0, bh = B;  // largest b with UB * prefix[b] <= x
+    while (bh - bl > 1) {
+      const int mid = (bl + bh) >> 1;
+      if ((long long)UB * prefix[mid] <= x) bl = mid; else bh = mid;
+    }
+    const long long nt = prefix[bl + 1] - prefix[bl];
+    const long long off = x - (long long)UB * prefix[bl];
+    const long long r = fdiv(off, nt), t = off - r * nt;
+    const long long F = (long long)UB * (prefix[bl] + kSwitchTiles * bl) + r * (nt + kSwitchTiles) + t;
+    const long long c = fdiv((F + 1) * P - 1, Ctot);
+    return c < P - 1 ? c : P - 1;
+  }
+};
+
 // (m, l) of partials c0 .. c0+n-1 of one unit into shared memory, every load
 // in flight at once; heads >= Gu and CTAs whose range is empty get (-inf, 0).
-__device__ __forceinline__ void stage_ml(const float* slot_ml, long long c0, int n, long long parts,
-                                         long long T, long long unit, int Gu, float* sm, float* sl) {
+__device__ __forceinline__ void stage_ml(const float* slot_ml, long long c0, int n, const Split& sp,
+                                         long long unit, int Gu, float* sm, float* sl) {
   for (int i = threadIdx.x; i < n * kMaxGroup; i += kCThreads) {
     const long long c = c0 + i / kMaxGroup;
     const int hd = i % kMaxGroup;
     float2 ml = make_float2(-INFINITY, 0.0f);
-    if (hd < Gu && c * T / parts != (c + 1) * T / parts)
+    if (hd < Gu && !sp.empty(c))
       ml = __ldcg(reinterpret_cast<const float2*>(slot_ml + ((c + unit) * kMaxGroup + hd) * 2));
     sm[i] = ml.x;
     sl[i] = ml.y;
@@ -351,22 +449,23 @@ __device__ __forceinline__ void stage_ml(const float* slot_ml, long long c0, int
 
 // Per-head (M, L) = (max m, sum l * 2^(m - M)) over the partials c_first ..
 // c_last of one unit.  Partials are staged kMergeChunk at a time; thread t
-// folds head t % 8 of every (kCThreads/8)-th staged partial, then the running
-// pairs of a head are combined, all in a fixed order.  On return sm/sl hold
-// the last staged chunk.
+// of the first kFold folds head t % 8 of every (kFold/8)-th staged partial,
+// then the running pairs of a head are combined, all in a fixed order.  On
+// return sm/sl hold the last staged chunk.
 __device__ __forceinline__ void unit_stats(const float* slot_ml, long long c_first, long long c_last,
-                                           long long parts, long long T, long long unit, int Gu,
+                                           const Split& sp, long long unit, int Gu,
                                            float* sm, float* sl, float* red_m, float* red_l,
                                            float* outM, float* outL) {
-  constexpr int J = kCThreads / kMaxGroup;
+  constexpr int kFold = kCThreads < 128 ? kCThreads : 128;  // threads that fold
+  constexpr int J = kFold / kMaxGroup;
   const int tid = threadIdx.x, hd = tid % kMaxGroup, j = tid / kMaxGroup;
   float m = -INFINITY, l = 0.0f;
   for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
     const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
     consumer_sync();  // the previous chunk has been folded
-    stage_ml(slot_ml, c0, n, parts, T, unit, Gu, sm, sl);
+    stage_ml(slot_ml, c0, n, sp, unit, Gu, sm, sl);
     consumer_sync();
-    for (int k = j; k < n; k += J) {
+    for (int k = j; tid < kFold && k < n; k += J) {
       const float mc = sm[k * kMaxGroup + hd], lc = sl[k * kMaxGroup + hd];
       if (mc == -INFINITY) continue;
       if (mc > m) {
@@ -429,12 +528,13 @@ __device__ __forceinline__ Segment locate(long long x, long long hi, const int* 
 // --------------------------------------------------------------- the kernel --
 
 template <int KB, int VB, int NB, int MODE, int GQ>
-__global__ void __launch_bounds__(kThreads, NB == 1 ? TQ_DECODE_MIN_CTAS : 2)
+__global__ void __launch_bounds__(kThreads, NB == 1 ? TQ_DECODE_MIN_CTAS : TQ_DECODE_MIN_CTAS_WIDE)
 decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   using SM = Smem<KB, VB, NB, MODE>;
   constexpr int D = SM::D;
   constexpr bool HASK = SM::kHasK, HASV = SM::kHasV;
   constexpr int KBB = Fmt<KB>::kBlockBytes, VBB = Fmt<VB>::kBlockBytes;
+  constexpr int kDepth = SM::kDepth;
   // GQ == 4 (at most four query heads per unit): score columns 4..7 repeat
   // heads 0..3, and the V products use the eight MMA columns as (head, dim
   // parity) pairs, so V fragments come straight from the table.  GQ == 8:
@@ -531,7 +631,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     if (tid == kThreads - 1) prefix[B] = run;
     __syncthreads();
   }
-  const long long T = (long long)prefix[p.batch] * UB;
+  const Split sp(prefix, p.batch, UB, gridDim.x);  // this launch's split
+  const long long T = sp.T;
 
   // ---- zero rows of empty sequences (only the V-producing passes) ---------
   if constexpr (MODE != kScores) {
@@ -545,13 +646,172 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   }
   if (T == 0) return;
 
-  const long long P = gridDim.x;
-  const long long lo = (long long)blockIdx.x * T / P;
-  const long long hi = ((long long)blockIdx.x + 1) * T / P;
-  auto cta_of = [&](long long x, long long parts) { return ((x + 1) * parts + T - 1) / T - 1; };
+  const long long lo = sp.start(blockIdx.x), hi = sp.start(blockIdx.x + 1);
   const int cw = warp;
   uint8_t* wring = ring + (size_t)cw * kDepth * SM::kSlotBytes;  // this warp's ring
   const uint32_t wring_s = smem_addr(wring);
+  // ---- query preparation: qhat = H.(s o q) (D1), as this lane's fp16 MMA
+  // B fragments plus the per-column score multipliers.  One warp per head
+  // row: lane l holds dims 4l..4l+3 of every 128-block, the butterflies of
+  // stride 1 and 2 are in-lane, strides 4..64 cross lanes.  Uses res as
+  // scratch.
+  auto prep_q = [&](int b, int h0, int Gu, uint32_t (&qf)[NB][8][2], float (&qmul)[2]) {
+    constexpr int kQRows = kDup ? 4 : kMaxGroup;
+    float* qs = res;  // [kQRows][D] scaled qhat
+    for (int j = cw; j < kQRows; j += kCWarps) {
+      float v[NB][4];
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        const size_t qi = ((size_t)b * p.q_heads + h0 + j) * D + blk * kBlock + 4 * lane;
+        if (j >= Gu) {
+          v[blk][0] = v[blk][1] = v[blk][2] = v[blk][3] = 0.0f;
+        } else if (p.q_f16) {
+          const uint2 h = *reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(p.q) + qi);
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+          const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+          v[blk][0] = a.x; v[blk][1] = a.y; v[blk][2] = c.x; v[blk][3] = c.y;
+        } else {
+          const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.q) + qi);
+          v[blk][0] = a.x; v[blk][1] = a.y; v[blk][2] = a.z; v[blk][3] = a.w;
+        }
+        const uint32_t sgn = p.sign_mask[lane >> 3] >> (4 * (lane & 7));  // signs of dims 4l..4l+3
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if ((sgn >> k) & 1u) v[blk][k] = -v[blk][k];
+      }
+      wht_rows<NB>(v, lane);
+      // power-of-two scale per head so fp16 fragments neither overflow nor
+      // fall into subnormals
+      float mx = 0.0f;
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx = fmaxf(mx, fabsf(v[blk][k]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const int qe = (mx > 0.0f) ? (ilogbf(mx) - 13) : 0;
+      if (lane == 0) qexp[j] = qe;
+      const float sc = ldexpf(1.0f, -qe);
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk)
+        *reinterpret_cast<float4*>(qs + j * D + blk * kBlock + 4 * lane) =
+            make_float4(v[blk][0] * sc, v[blk][1] * sc, v[blk][2] * sc, v[blk][3] * sc);
+    }
+    consumer_sync();
+    const int hr = kDup ? (R & 3) : R;  // this lane's score column's head
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float* q4 = qs + hr * D + blk * kBlock + 32 * g + 4 * j;
+        qf[blk][j][0] = pack_half2(q4[0], q4[1]);
+        qf[blk][j][1] = pack_half2(q4[2], q4[3]);
+      }
+    }
+    qmul[0] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g) & 3 : 2 * g]);
+    qmul[1] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g + 1) & 3 : 2 * g + 1]);
+    consumer_sync();  // res and qexp are reused after this
+  };
+
+  // ---- D7/D8: a unit's output from res, one inverse rotation per head,
+  // o = s o (H.acc) / L ---------------------------------------------------------
+  auto emit = [&](const Segment& sg) {
+    const int Gu = sg.Gu, b = sg.b, h0 = sg.h0;
+    const uint32_t sgn = p.sign_mask[lane >> 3] >> (4 * (lane & 7));  // signs of dims 4l..4l+3
+    for (int hd = cw; hd < Gu; hd += kCWarps) {  // one warp per head row
+      float v[NB][4];
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+        const float4 a = *reinterpret_cast<const float4*>(res + hd * D + blk * kBlock + 4 * lane);
+        v[blk][0] = a.x; v[blk][1] = a.y; v[blk][2] = a.z; v[blk][3] = a.w;
+      }
+      wht_rows<NB>(v, lane);
+      const float L = (MODE == kFused) ? u_L[hd] : 1.0f;
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if constexpr (MODE == kFused) v[blk][k] = v[blk][k] / L;
+          if ((sgn >> k) & 1u) v[blk][k] = -v[blk][k];
+        }
+        *reinterpret_cast<float4*>(p.out + ((size_t)b * p.q_heads + h0 + hd) * D + blk * kBlock + 4 * lane) =
+            make_float4(v[blk][0], v[blk][1], v[blk][2], v[blk][3]);
+      }
+    }
+  };
+
+  // ---- every partial of a unit merged into res (and u_M, u_L) in a fixed
+  // order; the unit's ticket is cleared for the next launch -------------------
+  auto merge_unit = [&](const Segment& sg) {
+    const int Gu = sg.Gu, unit = sg.unit, nt = sg.nt;
+    const long long Su = sg.Su;
+    __threadfence();
+    const long long c_first = sp.part_of(Su), c_last = sp.part_of(Su + nt - 1);
+    if constexpr (HASK) unit_stats(p.slot_ml, c_first, c_last, sp, unit, Gu, fac, stl, red_m, red_l, u_M, u_L);
+    for (int i = tid; i < Gu * D; i += kCThreads) res[i] = 0.0f;
+    const bool one_chunk = c_last - c_first < kMergeChunk;
+    for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
+      const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
+      // weights 2^(m_c - M) of this chunk's partials (0 for empty ranges;
+      // without scores, 1 for every non-empty range)
+      if constexpr (HASK) {
+        if (!one_chunk) {  // else unit_stats left this chunk staged
+          consumer_sync();
+          stage_ml(p.slot_ml, c0, n, sp, unit, Gu, fac, stl);
+          consumer_sync();
+        }
+        for (int i = tid; i < n * kMaxGroup; i += kCThreads) {
+          const float mc = fac[i];
+          fac[i] = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[i % kMaxGroup]);
+        }
+      } else {
+        consumer_sync();
+        for (int i = tid; i < n * kMaxGroup; i += kCThreads) {
+          const long long c = c0 + i / kMaxGroup;
+          fac[i] = (i % kMaxGroup < Gu && !sp.empty(c)) ? 1.0f : 0.0f;
+        }
+      }
+      consumer_sync();
+      // four consecutive dims per thread, many partials in flight (the
+      // merge is on the critical path of the whole launch)
+      for (int i = tid; i < Gu * D / 4; i += kCThreads) {
+        const int hd = (4 * i) / D, d = (4 * i) % D;
+        const float4* src =
+            reinterpret_cast<const float4*>(p.slot_acc + ((c0 + unit) * kMaxGroup + hd) * D + d);
+        float4 sacc = reinterpret_cast<const float4*>(res)[i];
+#pragma unroll 16
+        for (int cc = 0; cc < n; ++cc) {
+          const float f = fac[cc * kMaxGroup + hd];
+          const float4 a = __ldcg(src + (size_t)cc * kMaxGroup * D / 4);
+          if (f != 0.0f) {  // a partial that was never written may hold anything
+            sacc.x = fmaf(a.x, f, sacc.x);
+            sacc.y = fmaf(a.y, f, sacc.y);
+            sacc.z = fmaf(a.z, f, sacc.z);
+            sacc.w = fmaf(a.w, f, sacc.w);
+          }
+        }
+        reinterpret_cast<float4*>(res)[i] = sacc;
+      }
+    }
+    consumer_sync();
+    if (tid == 0) p.tickets[unit] = 0u;
+    consumer_sync();
+  };
+
+  // ---- add a segment's tiles to its unit's count: true for the CTA that
+  // completes it ------------------------------------------------------------------
+  auto count_tiles = [&](const Segment& sg) -> bool {
+    __threadfence();
+    consumer_sync();
+    if (tid == 0) {
+      const unsigned add = (unsigned)(sg.seg_hi - sg.seg_lo);
+      const unsigned old = atomicAdd(p.tickets + sg.unit, add);
+      flag[0] = (old + add == (unsigned)sg.nt) ? 1 : 0;
+    }
+    consumer_sync();
+    return flag[0] != 0;
+  };
+
   for (long long x = lo; x < hi;) {
     const Segment sg = locate(x, hi, prefix, p.batch, UB, n_hg, G, p.seq_cap, p.seq_lens);
     const int b = sg.b, nt = sg.nt, unit = sg.unit, h0 = sg.h0, Gu = sg.Gu, len = sg.len;
@@ -563,66 +823,77 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     const uint16_t* knp = p.k_norms + cache_row * NB;
     const uint16_t* vnp = p.v_norms + cache_row * NB;
 
-    // ---- per-unit query preparation: qhat = H.(s o q) (D1) ----------------
+    // Copy tile `tile` of this unit into ring slot `slot` (all lanes; one
+    // commit group).  Bytes past the end of the sequence are zero-filled.
+    auto issue = [&](int tile, int slot) {
+      const int t0 = tile * kTile;
+      const int nval = min(kTile, len - t0);  // >= 1
+      const bool full = nval == kTile;
+      const uint32_t sb = wring_s + (uint32_t)(slot * SM::kSlotBytes);
+      if constexpr (HASK) {
+        constexpr int kChunks = kTile * NB * KB;  // 16-byte chunks (KBB = 16 * KB)
+        constexpr int kPerTok = NB * KB;
+        const uint8_t* src = kcp + (size_t)t0 * NB * KBB;
+#pragma unroll
+        for (int c0 = 0; c0 < kChunks; c0 += 32) {
+          const int c = c0 + lane;
+          if (c < kChunks) {
+            const bool ok = full || c / kPerTok < nval;
+            cp_async16(sb + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
+          }
+        }
+        if (lane < 8 * NB) {  // norms: 4-byte pieces of the tile's 16*NB halves
+          const int e = 2 * lane;  // first half of the piece
+          const int valid = full ? 2 : max(0, min(2, nval * NB - e));
+          cp_async4(sb + SM::kOffSlotKN + 4u * lane, knp + (size_t)t0 * NB + (valid ? e : 0),
+                    2u * (uint32_t)valid);
+        }
+      }
+      if constexpr (HASV) {
+        constexpr int kChunks = kTile * NB * VB;
+        constexpr int kPerTok = NB * VB;
+        const uint8_t* src = vcp + (size_t)t0 * NB * VBB;
+#pragma unroll
+        for (int c0 = 0; c0 < kChunks; c0 += 32) {
+          const int c = c0 + lane;
+          if (c < kChunks) {
+            const bool ok = full || c / kPerTok < nval;
+            cp_async16(sb + SM::kOffSlotV + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
+          }
+        }
+        if (lane < 8 * NB) {
+          const int e = 2 * lane;
+          const int valid = full ? 2 : max(0, min(2, nval * NB - e));
+          cp_async4(sb + SM::kOffSlotVN + 4u * lane, vnp + (size_t)t0 * NB + (valid ? e : 0),
+                    2u * (uint32_t)valid);
+        }
+      }
+    };
+
+    // This lane's first K / V word inside a slot.
+    const int vlane = VB == 4 ? 8 * R : (VB == 3 ? 4 * ((3 * R) >> 1) : 4 * R);
+    const uint32_t koff = (uint32_t)((2 * R) * NB * KBB + g * KB * 4);
+    const uint32_t voff = (uint32_t)(SM::kOffSlotV + (4 * g) * NB * VBB + vlane);
+    // Warp cw takes tiles seg_lo + cw, seg_lo + cw + kCWarps, ...: tile i of
+    // the warp (i = 0, 1, ...) lives in slot i % kDepth.  The first kDepth
+    // copies are issued before the query preparation, which they overlap.
+    const int first = seg_lo + cw;
+    const int n_mine = first < seg_hi ? (seg_hi - first + kCWarps - 1) / kCWarps : 0;
+#pragma unroll
+    for (int i = 0; i < kDepth; ++i) {
+      if (i < n_mine) issue(first + i * kCWarps, i);
+      cp_async_commit();
+    }
+    // ---- per-unit query preparation ----------------------------------------
     uint32_t qf[NB][8][2];
     float qmul[2] = {0.0f, 0.0f};
     float lse2[2] = {0.0f, 0.0f};
-    if constexpr (HASK) {
-      float* qs = work;  // [8][D]
-      constexpr int kQRows = kDup ? 4 : kMaxGroup;
-      for (int i = tid; i < kQRows * D; i += kCThreads) {
-        const int j = i / D, d = i % D;
-        float v = 0.0f;
-        if (j < Gu) {
-          const size_t qi = ((size_t)b * p.q_heads + h0 + j) * D + d;
-          v = p.q_f16 ? __half2float(reinterpret_cast<const __half*>(p.q)[qi])
-                      : reinterpret_cast<const float*>(p.q)[qi];
-          const int e = d & (kBlock - 1);
-          if ((p.sign_mask[e >> 5] >> (e & 31)) & 1u) v = -v;
-        }
-        qs[i] = v;
-      }
-      consumer_sync();
-      for (int s = 1; s < kBlock; s <<= 1) {
-        for (int i = tid; i < kQRows * D / 2; i += kCThreads) {
-          const int j = i / (D / 2), rem = i % (D / 2);
-          const int a = (rem / s) * 2 * s + (rem % s);
-          float* row = qs + j * D;
-          const float u = row[a], w = row[a + s];
-          row[a] = u + w;
-          row[a + s] = u - w;
-        }
-        consumer_sync();
-      }
-      // power-of-two scale per head so fp16 fragments neither overflow nor
-      // fall into subnormals
-      for (int j = cw; j < kQRows; j += kCWarps) {
-        float mx = 0.0f;
-        for (int d = lane; d < D; d += 32) mx = fmaxf(mx, fabsf(qs[j * D + d]));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) qexp[j] = (mx > 0.0f) ? (ilogbf(mx) - 13) : 0;
-      }
-      consumer_sync();
-      const float qsc = ldexpf(1.0f, -qexp[kDup ? (R & 3) : R]);
-#pragma unroll
-      for (int blk = 0; blk < NB; ++blk) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float* q4 = qs + (kDup ? (R & 3) : R) * D + blk * kBlock + 32 * g + 4 * j;
-          qf[blk][j][0] = pack_half2(q4[0] * qsc, q4[1] * qsc);
-          qf[blk][j][1] = pack_half2(q4[2] * qsc, q4[3] * qsc);
-        }
-      }
-      qmul[0] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g) & 3 : 2 * g]);
-      qmul[1] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g + 1) & 3 : 2 * g + 1]);
-      consumer_sync();  // work area is reused below
-    }
+    if constexpr (HASK) prep_q(b, h0, Gu, qf, qmul);
     if constexpr (MODE == kSparseV) {
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote
-      const long long P1 = p1_ctas;
-      unit_stats(p.slot_ml, cta_of(Su, P1), cta_of(Su + nt - 1, P1), P1, T, unit, Gu, fac, stl, red_m, red_l,
+      const Split sp1(prefix, p.batch, UB, p1_ctas);
+      unit_stats(p.slot_ml, sp1.part_of(Su), sp1.part_of(Su + nt - 1), sp1, unit, Gu, fac, stl, red_m, red_l,
                  u_M, u_L);
       if (tid < Gu) u_lse[tid] = u_M[tid] + __log2f(u_L[tid]);
       consumer_sync();
@@ -819,66 +1090,6 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     };
 
     {
-      // Copy tile `tile` of this unit into ring slot `slot` (all lanes; one
-      // commit group).  Bytes past the end of the sequence are zero-filled.
-      auto issue = [&](int tile, int slot) {
-        const int t0 = tile * kTile;
-        const int nval = min(kTile, len - t0);  // >= 1
-        const bool full = nval == kTile;
-        const uint32_t sb = wring_s + (uint32_t)(slot * SM::kSlotBytes);
-        if constexpr (HASK) {
-          constexpr int kChunks = kTile * NB * KB;  // 16-byte chunks (KBB = 16 * KB)
-          constexpr int kPerTok = NB * KB;
-          const uint8_t* src = kcp + (size_t)t0 * NB * KBB;
-#pragma unroll
-          for (int c0 = 0; c0 < kChunks; c0 += 32) {
-            const int c = c0 + lane;
-            if (c < kChunks) {
-              const bool ok = full || c / kPerTok < nval;
-              cp_async16(sb + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
-            }
-          }
-          if (lane < 8 * NB) {  // norms: 4-byte pieces of the tile's 16*NB halves
-            const int e = 2 * lane;  // first half of the piece
-            const int valid = full ? 2 : max(0, min(2, nval * NB - e));
-            cp_async4(sb + SM::kOffSlotKN + 4u * lane, knp + (size_t)t0 * NB + (valid ? e : 0),
-                      2u * (uint32_t)valid);
-          }
-        }
-        if constexpr (HASV) {
-          constexpr int kChunks = kTile * NB * VB;
-          constexpr int kPerTok = NB * VB;
-          const uint8_t* src = vcp + (size_t)t0 * NB * VBB;
-#pragma unroll
-          for (int c0 = 0; c0 < kChunks; c0 += 32) {
-            const int c = c0 + lane;
-            if (c < kChunks) {
-              const bool ok = full || c / kPerTok < nval;
-              cp_async16(sb + SM::kOffSlotV + 16u * c, src + (ok ? 16 * c : 0), ok ? 16u : 0u);
-            }
-          }
-          if (lane < 8 * NB) {
-            const int e = 2 * lane;
-            const int valid = full ? 2 : max(0, min(2, nval * NB - e));
-            cp_async4(sb + SM::kOffSlotVN + 4u * lane, vnp + (size_t)t0 * NB + (valid ? e : 0),
-                      2u * (uint32_t)valid);
-          }
-        }
-      };
-
-      // This lane's first K / V word inside a slot.
-      const int vlane = VB == 4 ? 8 * R : (VB == 3 ? 4 * ((3 * R) >> 1) : 4 * R);
-      const uint32_t koff = (uint32_t)((2 * R) * NB * KBB + g * KB * 4);
-      const uint32_t voff = (uint32_t)(SM::kOffSlotV + (4 * g) * NB * VBB + vlane);
-      // Warp cw takes tiles seg_lo + cw, seg_lo + cw + kCWarps, ...: tile i of
-      // the warp (i = 0, 1, ...) lives in slot i % kDepth.
-      const int first = seg_lo + cw;
-      const int n_mine = first < seg_hi ? (seg_hi - first + kCWarps - 1) / kCWarps : 0;
-#pragma unroll
-      for (int i = 0; i < kDepth; ++i) {
-        if (i < n_mine) issue(first + i * kCWarps, i);
-        cp_async_commit();
-      }
       // Tile i of the warp sits in slot i % kDepth.  Once both halves of a
       // tile are in registers, its slot is handed to tile i + kDepth, so the
       // copy runs under the tile's arithmetic.
@@ -983,11 +1194,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     consumer_sync();
 
     const bool whole = (seg_lo == 0 && seg_hi == nt);
-    bool finalize = false;
     if (whole && MODE != kScores) {
-      finalize = true;  // this CTA saw the entire unit: no partial needed
+      emit(sg);  // this CTA saw the entire unit: no partial needed
     } else {
-      // ---- publish the partial, count tiles, the last CTA merges ----------
+      // ---- publish the partial ---------------------------------------------
       const long long slot = blockIdx.x + unit;
       if constexpr (HASK) {
         if (tid < Gu) {
@@ -1000,97 +1210,16 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           p.slot_acc[(slot * kMaxGroup + i / D) * D + i % D] = res[i];
       }
       if constexpr (MODE != kScores) {
-        __threadfence();
-        consumer_sync();
-        if (tid == 0) {
-          const unsigned add = (unsigned)(seg_hi - seg_lo);
-          const unsigned old = atomicAdd(p.tickets + unit, add);
-          flag[0] = (old + add == (unsigned)nt) ? 1 : 0;
+        if (count_tiles(sg)) {  // the last CTA of the unit merges its partials
+          merge_unit(sg);
+          emit(sg);
         }
-        consumer_sync();
-        finalize = flag[0] != 0;
-        if (finalize) {
-          __threadfence();
-          const long long c_first = cta_of(Su, P), c_last = cta_of(Su + nt - 1, P);
-          if constexpr (HASK)
-            unit_stats(p.slot_ml, c_first, c_last, P, T, unit, Gu, fac, stl, red_m, red_l, u_M, u_L);
-          for (int i = tid; i < Gu * D; i += kCThreads) res[i] = 0.0f;
-          const bool one_chunk = c_last - c_first < kMergeChunk;
-          for (long long c0 = c_first; c0 <= c_last; c0 += kMergeChunk) {
-            const int n = (int)min((long long)kMergeChunk, c_last - c0 + 1);
-            // weights 2^(m_c - M) of this chunk's partials (0 for empty ranges;
-            // without scores, 1 for every non-empty range)
-            if constexpr (HASK) {
-              if (!one_chunk) {  // else unit_stats left this chunk staged
-                consumer_sync();
-                stage_ml(p.slot_ml, c0, n, P, T, unit, Gu, fac, stl);
-                consumer_sync();
-              }
-              for (int i = tid; i < n * kMaxGroup; i += kCThreads) {
-                const float mc = fac[i];
-                fac[i] = (mc == -INFINITY) ? 0.0f : ex2(mc - u_M[i % kMaxGroup]);
-              }
-            } else {
-              consumer_sync();
-              for (int i = tid; i < n * kMaxGroup; i += kCThreads) {
-                const long long c = c0 + i / kMaxGroup;
-                fac[i] = (i % kMaxGroup < Gu && c * T / P != (c + 1) * T / P) ? 1.0f : 0.0f;
-              }
-            }
-            consumer_sync();
-            // four consecutive dims per thread, many partials in flight (the
-            // merge is on the critical path of the whole launch)
-            for (int i = tid; i < Gu * D / 4; i += kCThreads) {
-              const int hd = (4 * i) / D, d = (4 * i) % D;
-              const float4* src =
-                  reinterpret_cast<const float4*>(p.slot_acc + ((c0 + unit) * kMaxGroup + hd) * D + d);
-              float4 sacc = reinterpret_cast<const float4*>(res)[i];
-#pragma unroll 16
-              for (int cc = 0; cc < n; ++cc) {
-                const float f = fac[cc * kMaxGroup + hd];
-                const float4 a = __ldcg(src + (size_t)cc * kMaxGroup * D / 4);
-                if (f != 0.0f) {  // a partial that was never written may hold anything
-                  sacc.x = fmaf(a.x, f, sacc.x);
-                  sacc.y = fmaf(a.y, f, sacc.y);
-                  sacc.z = fmaf(a.z, f, sacc.z);
-                  sacc.w = fmaf(a.w, f, sacc.w);
-                }
-              }
-              reinterpret_cast<float4*>(res)[i] = sacc;
-            }
-          }
-          consumer_sync();
-          if (tid == 0) p.tickets[unit] = 0u;
-          consumer_sync();
-        }
-      }
-    }
-
-    if (finalize) {
-      // ---- D7/D8: one inverse rotation per head, o = s o (H.acc) / L -----
-      for (int s = 1; s < kBlock; s <<= 1) {
-        for (int i = tid; i < Gu * D / 2; i += kCThreads) {
-          const int hd = i / (D / 2), rem = i % (D / 2);
-          const int a = (rem / s) * 2 * s + (rem % s);
-          float* row = res + hd * D;
-          const float u = row[a], w = row[a + s];
-          row[a] = u + w;
-          row[a + s] = u - w;
-        }
-        consumer_sync();
-      }
-      for (int i = tid; i < Gu * D; i += kCThreads) {
-        const int hd = i / D, d = i % D;
-        const int e = d & (kBlock - 1);
-        float v = res[i];
-        if constexpr (MODE == kFused) v = v / u_L[hd];
-        if ((p.sign_mask[e >> 5] >> (e & 31)) & 1u) v = -v;
-        p.out[((size_t)b * p.q_heads + h0 + hd) * D + d] = v;
       }
     }
     consumer_sync();
     x = Su + seg_hi;
   }
+
 }
 
 // --------------------------------------------------------------- launching --

@@ -69,6 +69,19 @@ def test_decode_bit_widths(kb, vb, d):
     _run(w)
 
 
+@pytest.mark.parametrize("kb,vb", [(4, 4), (3, 4), (4, 2)])
+@pytest.mark.parametrize("hq", [8, 16])
+def test_decode_wide_head_fused_bit_widths(kb, vb, hq):
+    # head_dim 256 with sparse-V off: the fused kernel with the largest ring
+    # slots (the ring is shortened to fit shared memory); groups of 2 and 4
+    w = inputs.make("ragged", batch=2, seq=700)
+    rng = np.random.default_rng(7 * kb + vb + hq)
+    w.k_bits, w.v_bits, w.q_heads = kb, vb, hq
+    w.seq_lens = np.array([700, 333], dtype=np.int32)
+    w.q = rng.standard_normal((2, hq, 256)).astype(np.float16)
+    _run(w, sparse_thr=0.0)
+
+
 @pytest.mark.parametrize("hq,hkv", [(2, 2), (6, 2), (16, 2), (24, 2), (20, 4)])
 def test_decode_group_sizes(hq, hkv):
     w = inputs.make("gqa", batch=2, seq=200)
