@@ -11,6 +11,8 @@
 // them on packed f32x2 arithmetic), the seventh pairs the two lanes through
 // one shuffle per element.  A lane's 64 codes are contiguous in the packed
 // bitstream (8*b bytes at byte 8*b*h), so stores are plain vector stores.
+// For fp16 input the random signs are applied to the fp16 sign bits as the
+// elements are converted (one XOR per element pair).
 
 #include <cuda_fp16.h>
 
@@ -48,7 +50,7 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t (&w)[2 
 }
 
 template <int BITS, bool F16, int SIDE>
-__device__ __forceinline__ void encode_side(const EncodeParams& p) {
+__device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* warp_signs) {
   constexpr int L = 1 << BITS;
   constexpr int NPOS = L / 2 - 1;  // positive decision boundaries
   const void* in = p.in[SIDE];
@@ -78,10 +80,25 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p) {
   if constexpr (F16) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(in) +
                                                       (row * p.head_dim + j * kBlock + 64 * h));
+    uint4 raw[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) raw[c] = ok ? __ldcs(src + c) : make_uint4(0, 0, 0, 0);
+    // s o x (E1) on the fp16 bits, one mask word per element pair: word m of
+    // half hh holds s_(64hh+2m) in bit 15 and s_(64hh+2m+1) in bit 31.  Each
+    // warp builds its own copy while its loads are in flight.
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t wd = p.sign_mask[2 * hh + (lane >> 4)];
+      const int bit = (2 * lane) & 31;
+      warp_signs[hh * 32 + lane] = (((wd >> bit) & 1u) << 15) | (((wd >> (bit + 1)) & 1u) << 31);
+    }
+    __syncwarp();
+    const uint4* sgn = reinterpret_cast<const uint4*>(warp_signs + 32 * h);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      uint4 v = ok ? __ldcs(src + c) : make_uint4(0, 0, 0, 0);
-      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      const uint4 v = raw[c];
+      const uint4 mk = sgn[c];
+      const uint32_t wv[4] = {v.x ^ mk.x, v.y ^ mk.y, v.z ^ mk.z, v.w ^ mk.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         __half2 hv = *reinterpret_cast<const __half2*>(&wv[e]);
@@ -111,8 +128,8 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p) {
   ss += __shfl_xor_sync(0xffffffffu, ss, 1);
   const float n = __fsqrt_rn(ss);
 
-  // ---- sign flip (E1): s o x ---------------------------------------------
-  {
+  // ---- sign flip (E1): s o x (fp32 input; fp16 input was flipped on load)
+  if constexpr (!F16) {
     const uint32_t w0 = h ? p.sign_mask[2] : p.sign_mask[0];
     const uint32_t w1 = h ? p.sign_mask[3] : p.sign_mask[1];
 #pragma unroll
@@ -195,10 +212,12 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p) {
 
 template <int KB, int VB, bool F16>
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_constant__ EncodeParams p) {
+  __shared__ __align__(16) uint32_t signs[kEncThreads / 32][64];  // per-warp fp16 sign masks
+  uint32_t* ws = signs[threadIdx.x >> 5];
   if (blockIdx.y == 0) {
-    if (p.in[0]) encode_side<KB, F16, 0>(p);
+    if (p.in[0]) encode_side<KB, F16, 0>(p, ws);
   } else {
-    if (p.in[1]) encode_side<VB, F16, 1>(p);
+    if (p.in[1]) encode_side<VB, F16, 1>(p, ws);
   }
 }
 
