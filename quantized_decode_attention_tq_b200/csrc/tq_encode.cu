@@ -6,13 +6,15 @@
 // TurboQuant article §3.2 (H_random from a random +-1 diagonal and the
 // Hadamard matrix, fast transform in O(d log d)) and §3.3 (Lloyd-Max).
 //
-// Mapping: two lanes per 128-block, lane h holding elements [64h, 64h+64)
-// as 32 float2 registers.  Six butterfly stages run in registers (five of
-// them on packed f32x2 arithmetic), the seventh pairs the two lanes through
-// one shuffle per element.  A lane's 64 codes are contiguous in the packed
-// bitstream (8*b bytes at byte 8*b*h), so stores are plain vector stores.
-// For fp16 input the random signs are applied to the fp16 sign bits as the
-// elements are converted (one XOR per element pair).
+// Mapping: two lanes per 128-block.  The block is 16 chunks of 8 elements;
+// lane h holds chunks 2c + h (c = 0..7) as 32 float2 registers, so a lane
+// pair reads 32 contiguous bytes per fp16 load.  The butterfly stages commute,
+// so the six whose partners share a lane run in registers (five of them on
+// packed f32x2 arithmetic) and the stride-8 stage pairs the two lanes through
+// one shuffle per element.  Lane 0 stores chunks 0..7 of the packed bitstream
+// and lane 1 chunks 8..15 (8*b bytes each, plain vector stores) after the
+// pair swaps four chunk words.  For fp16 input the random signs are applied
+// to the fp16 sign bits as the elements are converted (one XOR per pair).
 
 #include <cuda_fp16.h>
 
@@ -78,18 +80,22 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
   // ---- load 64 elements (E1), convert to fp32 --------------------------
   float2 x[32];
   if constexpr (F16) {
+    // chunk 2c + h of the block (8 elements, 16 B): a lane pair reads 32
+    // contiguous bytes per load
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(in) +
-                                                      (row * p.head_dim + j * kBlock + 64 * h));
+                                                      (row * p.head_dim + j * kBlock)) + h;
     uint4 raw[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) raw[c] = ok ? __ldcs(src + c) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < 8; ++c) raw[c] = ok ? __ldcs(src + 2 * c) : make_uint4(0, 0, 0, 0);
     // s o x (E1) on the fp16 bits, one mask word per element pair: word m of
-    // half hh holds s_(64hh+2m) in bit 15 and s_(64hh+2m+1) in bit 31.  Each
-    // warp builds its own copy while its loads are in flight.
+    // lane half hh covers elements i, i+1 with i = 16(m/4) + 8hh + 2(m%4),
+    // s_i in bit 15 and s_(i+1) in bit 31.  Each warp builds its own copy
+    // while its loads are in flight.
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t wd = p.sign_mask[2 * hh + (lane >> 4)];
-      const int bit = (2 * lane) & 31;
+      const int i = 16 * (lane >> 2) + 8 * hh + 2 * (lane & 3);
+      const uint32_t wd = p.sign_mask[i >> 5];
+      const int bit = i & 31;
       warp_signs[hh * 32 + lane] = (((wd >> bit) & 1u) << 15) | (((wd >> (bit + 1)) & 1u) << 31);
     }
     __syncwarp();
@@ -107,12 +113,15 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
     }
   } else {
     const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(in) +
-                                                        (row * p.head_dim + j * kBlock + 64 * h));
+                                                        (row * p.head_dim + j * kBlock + 8 * h));
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      float4 v = ok ? __ldcs(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      x[2 * c] = make_float2(v.x, v.y);
-      x[2 * c + 1] = make_float2(v.z, v.w);
+    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float4 v = ok ? __ldcs(src + 4 * c + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[4 * c + 2 * q] = make_float2(v.x, v.y);
+        x[4 * c + 2 * q + 1] = make_float2(v.z, v.w);
+      }
     }
   }
 
@@ -130,14 +139,16 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
 
   // ---- sign flip (E1): s o x (fp32 input; fp16 input was flipped on load)
   if constexpr (!F16) {
-    const uint32_t w0 = h ? p.sign_mask[2] : p.sign_mask[0];
-    const uint32_t w1 = h ? p.sign_mask[3] : p.sign_mask[1];
+    // element (c, e) of the lane is i = 16c + 8h + e: sign word c/2, bit
+    // 16(c%2) + 8h + e
+    uint32_t sw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sw[q] = p.sign_mask[q] >> (8 * h);
 #pragma unroll
     for (int m = 0; m < 32; ++m) {
-      const uint32_t w = (m < 16) ? w0 : w1;
-      const int bit = (2 * m) & 31;
-      x[m].x = apply_sign(x[m].x, w, bit);
-      x[m].y = apply_sign(x[m].y, w, bit + 1);
+      const int c = m >> 2, bit = 16 * (c & 1) + 2 * (m & 3);
+      x[m].x = apply_sign(x[m].x, sw[c >> 1], bit);
+      x[m].y = apply_sign(x[m].y, sw[c >> 1], bit + 1);
     }
   }
 
@@ -155,7 +166,7 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
       }
     }
   }
-  {  // stride 64: the partner lane holds the other half of the block.
+  {  // stride 8: the partner lane holds the other chunks of the block.
     const float sg = h ? -1.0f : 1.0f;
     const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
@@ -177,9 +188,11 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
 #pragma unroll
   for (int k = 0; k < NPOS; ++k) thr[k] = p.pos_bounds[SIDE][k] * n;
 
-  uint32_t w[2 * BITS];
+  // Codes of the lane's chunk c (8 codes, 8*BITS bits) in g[c]; chunk c of
+  // lane h is chunk 2c + h of the block.
+  uint32_t g[8];
 #pragma unroll
-  for (int k = 0; k < 2 * BITS; ++k) w[k] = 0;
+  for (int c = 0; c < 8; ++c) g[c] = 0;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     const float y = (i & 1) ? x[i >> 1].y : x[i >> 1].x;
@@ -189,11 +202,26 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
     for (int k = 0; k < NPOS; ++k) m += (a > thr[k]) ? 1 : 0;
     const int lowside = L / 2 - 1 - m;
     const uint32_t idx = (uint32_t)(y > 0.0f ? (lowside ^ (L - 1)) : lowside);
-    // ---- pack (E5): LSB-first bitstream --------------------------------
-    const int bit = BITS * i;
+    g[i >> 3] |= idx << (BITS * (i & 7));
+  }
+  // ---- pack (E5): LSB-first bitstream.  Lane 0 stores chunks 0..7, lane 1
+  // chunks 8..15; the pair swaps the four chunk words each needs.
+  uint32_t grp[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t r = __shfl_xor_sync(0xffffffffu, h ? g[q] : g[4 + q], 1);
+    grp[2 * q] = h ? r : g[q];
+    grp[2 * q + 1] = h ? g[4 + q] : r;
+  }
+  uint32_t w[2 * BITS];
+#pragma unroll
+  for (int k = 0; k < 2 * BITS; ++k) w[k] = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int bit = 8 * BITS * q;
     const int wi = bit >> 5, sh = bit & 31;
-    w[wi] |= idx << sh;
-    if (sh + BITS > 32) w[wi + 1] |= idx >> (32 - sh);
+    w[wi] |= grp[q] << sh;
+    if (sh + 8 * BITS > 32) w[wi + 1] |= grp[q] >> (32 - sh);
   }
 
   if (ok) {
