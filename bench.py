@@ -2,11 +2,12 @@
 """Benchmark of the TurboQuant-style decode step on B200.
 
 One step = the hot path for one generated token of every sequence in the
-batch: encode the newest K/V row of each (batch, kv-head) into the packed cache
-(rotate, norm, quantise, pack) and run single-token decode attention over the
-whole cache (Q rotation, Hadamard-domain scores from codes, online softmax,
-rotated-domain V sum, split merge, inverse rotation).  The newest row is
-written at position seq_len - 1, so every step does identical work.
+batch, as one tq_decode_step launch (two with sparse-V): encode the newest K/V
+row of each (batch, kv-head) into the packed cache (rotate, norm, quantise,
+pack) and run single-token decode attention over the whole cache (Q rotation,
+Hadamard-domain scores from codes, online softmax, rotated-domain V sum, split
+merge, inverse rotation).  The newest row is written at position seq_len - 1,
+so every step does identical work.
 
 Default workload: GQA decode, B8, Hq32/Hkv8, D128, S32768, K3/V3, fp16 Q.
 The packed cache (210 MB) rotates over enough copies to exceed 3x L2, so no
@@ -85,7 +86,7 @@ def kv_bytes(w):
 def step_io_bytes(w):
     q = w.batch * w.q_heads * w.head_dim * np.dtype(w.dtype).itemsize
     kv_new = 2 * w.batch * w.kv_heads * w.head_dim * np.dtype(w.dtype).itemsize
-    lens = 2 * 4 * w.batch  # seq_lens and start positions
+    lens = 4 * w.batch  # seq_lens (the new token sits at seq_lens - 1)
     out = w.batch * w.q_heads * w.head_dim * 4
     return q + kv_new + lens, out
 
@@ -282,47 +283,41 @@ def run_tq(args):
     # step inputs: the newest row of every (batch, kv-head) and the query
     lens_np = w.seq_lens.astype(np.int32)
     pos_np = (lens_np - 1).astype(np.int32)
-    k_new_np = np.ascontiguousarray(w.k[np.arange(w.batch), :, pos_np][:, :, None, :])
-    v_new_np = np.ascontiguousarray(w.v[np.arange(w.batch), :, pos_np][:, :, None, :])
+    k_new_np = np.ascontiguousarray(w.k[np.arange(w.batch), :, pos_np])  # [B, Hkv, D]
+    v_new_np = np.ascontiguousarray(w.v[np.arange(w.batch), :, pos_np])
     q = torch.from_numpy(w.q).to(dev)
     k_new = torch.from_numpy(k_new_np).to(dev)
     v_new = torch.from_numpy(v_new_np).to(dev)
     lens = torch.from_numpy(lens_np).to(dev)
-    start = torch.from_numpy(pos_np).to(dev)
     out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float32, device=dev)
     ws = tq.alloc_workspace(desc, w.q_heads, w.sparse_thr, dev)
     decode_launches = 2 if w.sparse_thr > 0 else 1
 
-    def enc(c):
-        tq.encode_kv(caches[c], kcb, vcb, k_new, v_new, start_pos=start)
-
-    def dec(c):
-        tq.decode_attention(caches[c], kcb, vcb, q, lens, w.scale, out, ws, sparse_thr=w.sparse_thr)
+    def step(c):
+        # one decode step: the newest token of every sequence is encoded into
+        # the cache at lens - 1 inside the decode launch, then attended over
+        tq.decode_step(caches[c], kcb, vcb, q, k_new, v_new, lens, w.scale, out, ws,
+                       sparse_thr=w.sparse_thr)
 
     for c in range(n_copies):  # eager warm-up (also primes the launch caches)
-        enc(c)
-        dec(c)
+        step(c)
     torch.cuda.synchronize()
 
-    # ---- CUDA graphs: one for the encode launch, one for the decode launch(es)
-    g_enc, g_dec = [], []
+    # ---- CUDA graphs: one per cache copy, holding the step's launch(es) ------
+    g_step = []
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         for c in range(n_copies):
-            ge, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            with torch.cuda.graph(ge, stream=s):
-                enc(c)
-            with torch.cuda.graph(gd, stream=s):
-                dec(c)
-            g_enc.append(ge)
-            g_dec.append(gd)
+            gs = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gs, stream=s):
+                step(c)
+            g_step.append(gs)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
 
     for i in range(args.warmup):
-        g_enc[i % n_copies].replay()
-        g_dec[i % n_copies].replay()
+        g_step[i % n_copies].replay()
     torch.cuda.synchronize()
 
     # ---- timed region -------------------------------------------------------
@@ -337,10 +332,8 @@ def run_tq(args):
     time.sleep(0.3)
     ev0.record(stream)
     for i in range(args.steps):
-        c = i % n_copies
-        g_enc[c].replay()
         ea[i].record(stream)
-        g_dec[c].replay()
+        g_step[i % n_copies].replay()
         eb[i].record(stream)
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -356,7 +349,7 @@ def run_tq(args):
     # ---- end to end through the public API with host buffers ---------------
     h2d, d2h = step_io_bytes(w)
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
-    q_h, k_h, v_h, l_h, s_h = pin(w.q), pin(k_new_np), pin(v_new_np), pin(lens_np), pin(pos_np)
+    q_h, k_h, v_h, l_h = pin(w.q), pin(k_new_np), pin(v_new_np), pin(lens_np)
     out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
 
     def e2e_step(c):
@@ -364,9 +357,7 @@ def run_tq(args):
         k_new.copy_(k_h, non_blocking=True)
         v_new.copy_(v_h, non_blocking=True)
         lens.copy_(l_h, non_blocking=True)
-        start.copy_(s_h, non_blocking=True)
-        enc(c)
-        dec(c)
+        step(c)
         out_h.copy_(out, non_blocking=True)
 
     for i in range(max(3, args.warmup)):
@@ -387,7 +378,7 @@ def run_tq(args):
     encode_info = None
     if not args.no_encode and rank == 0:
         from quantized_decode_attention_tq_b200 import inputs
-        del caches, g_enc, g_dec
+        del caches, g_step
         torch.cuda.empty_cache()
         we = inputs.make("encode", with_q=False)
         de = tq.kv_desc(we.batch, we.kv_heads, we.head_dim, we.seq_cap, we.k_bits, we.v_bits)
@@ -448,7 +439,7 @@ def run_tq(args):
                          "algorithmic_bytes_per_launch": kvb},
             "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * (1 + decode_launches),
+            "gpu_launches": args.steps * decode_launches,
             "clocks": clocks,
             "encode": encode_info,
             "cpu_baseline": cpu,

@@ -177,6 +177,36 @@ int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const t
                         void* stream);
 
 /*
+ * tq_decode_step -- one decode step in one launch: append every sequence's
+ * new token to the cache, then attend over the cache including it.  In a
+ * decode step the new token's K/V rows are written into the quantised cache
+ * and flash attention then reads it (README backend table: turbo KV rows
+ * written by SET_ROWS, read by the flash-attention kernels); here both run in
+ * the same kernel.
+ *   - seq_lens counts the new token: for sequence b, rows k_new[b, h, :] and
+ *     v_new[b, h, :] are encoded exactly as tq_encode_kv would (block norm,
+ *     signs, WHT, codebook index, packing) and written at position
+ *     seq_lens[b] - 1, after seq_lens is clamped to [0, seq_cap]
+ *     (TQ_DEV_LEN_RANGE); a sequence of length 0 appends nothing.  Then the
+ *     output is that of tq_decode_attention over positions [0, seq_lens[b]).
+ *   - k_new, v_new: device [batch, kv_heads, head_dim], kv_dtype TQ_F32 or
+ *     TQ_F16, 16-byte aligned.  The norms and codes of the appended token
+ *     may differ from tq_encode_kv's by one fp16 ulp where the fp32 norm is
+ *     at an fp16 rounding midpoint, and by one code where a value is within
+ *     rounding of a decision boundary (the norm is summed in another order).
+ *   - With sparse_thr > 0 the step is two launches (the append rides in the
+ *     first, which scores K).
+ * Every other argument, limit and error is that of tq_decode_attention; the
+ * cache buffers are written as well as read.
+ */
+int tq_decode_step(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                   int q_heads, const void* q, int q_dtype, const void* k_new, const void* v_new,
+                   int kv_dtype, uint8_t* k_codes, uint16_t* k_norms, uint8_t* v_codes,
+                   uint16_t* v_norms, const int32_t* seq_lens, float scale, float sparse_thr,
+                   float* out, void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                   void* stream);
+
+/*
  * tq_decode_attention_noalloc -- tq_decode_attention for callers that must
  * not allocate device memory.  The pages have no counterpart: this is a
  * deployment variant of the same decode kernels, not a step of the method.

@@ -40,6 +40,10 @@ SIGNATURES = {
     "tq_decode_attention": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                                     c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "tq_decode_step": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
+                               c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_float, c_float, c_void_p, c_void_p, c_size_t, c_void_p,
+                               c_void_p]),
     "tq_decode_attention_noalloc": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p,
                                             c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_float, c_float, c_void_p, c_void_p, c_void_p]),

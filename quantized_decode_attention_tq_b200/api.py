@@ -138,6 +138,25 @@ def decode_attention(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, 
     return out
 
 
+def decode_step(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, k_new, v_new, seq_lens, scale: float,
+                out, workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """One decode step (tq_decode_step): write each sequence's new K/V row
+    [B, Hkv, D] at position seq_lens[b] - 1, then attend over the cache."""
+    if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    q_heads = q.shape[1]
+    st = lib().tq_decode_step(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb), q_heads,
+        _ptr(q, "q"), _dtype_code(q), _ptr(k_new, "k_new"), _ptr(v_new, "v_new"), _dtype_code(k_new),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_step", st)
+    return out
+
+
 def decode_attention_noalloc(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, scale: float,
                              out, sparse_thr: float = 0.0, status=None, stream=None):
     """Decode attention without a caller workspace (tq_decode_attention_noalloc).

@@ -371,6 +371,70 @@ __device__ __forceinline__ void wht_rows(float (&v)[NB][4], int lane) {
   }
 }
 
+// Decode step: encode 128-block `blk` of the new token's K (side 0) or V
+// (side 1) row `row` of kv_new into cache token `tok`, by one warp (lane l
+// holds elements 4l..4l+3).  Same steps as the encoder: fp16 block norm of
+// x, signs, unnormalised WHT, idx = #{boundaries < y / n} counted on |y|
+// against T_k * n, LSB-first packing ("TheTom/llama-cpp-turboquant" README,
+// table "量化类型"; intelliparadigm TurboQuant article §3.2-§3.3).  `stage`
+// is 16 words of this warp's shared memory.
+__device__ __noinline__ void append_block(const DecodeParams& p, int side, int blk, size_t row,
+                                          size_t tok, int lane, uint32_t* stage) {
+  const int bits = side ? p.v_bits : p.k_bits;
+  const int L = 1 << bits;
+  const int nb = p.head_dim / kBlock;
+  const size_t e0 = row * p.head_dim + (size_t)blk * kBlock + 4 * lane;
+  float v[1][4];
+  if (p.kv_new_f16) {
+    const uint2 h = *reinterpret_cast<const uint2*>(static_cast<const __half*>(p.kv_new[side]) + e0);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+    const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+    v[0][0] = a.x; v[0][1] = a.y; v[0][2] = c.x; v[0][3] = c.y;
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(p.kv_new[side]) + e0);
+    v[0][0] = a.x; v[0][1] = a.y; v[0][2] = a.z; v[0][3] = a.w;
+  }
+  float ss = v[0][0] * v[0][0];
+  ss = fmaf(v[0][1], v[0][1], ss);
+  ss = fmaf(v[0][2], v[0][2], ss);
+  ss = fmaf(v[0][3], v[0][3], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float n = __fsqrt_rn(ss);
+  const uint32_t sgn = p.sign_mask[lane >> 3] >> (4 * (lane & 7));
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if ((sgn >> k) & 1u) v[0][k] = -v[0][k];
+  wht_rows<1>(v, lane);
+  uint32_t field = 0;  // this lane's 4 codes, bits*4 bits
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float y = v[0][e], a = fabsf(y);
+    int m = 0;
+    for (int k = 0; k < L / 2 - 1; ++k) m += (a > p.pos_bounds[side][k] * n) ? 1 : 0;
+    const int lowside = L / 2 - 1 - m;
+    const uint32_t idx = (uint32_t)(y > 0.0f ? (lowside ^ (L - 1)) : lowside);
+    field |= idx << (bits * e);
+  }
+  // lane l's codes are bits [4*bits*l, 4*bits*(l+1)) of the block's stream
+  if (lane < 4 * bits) stage[lane] = 0u;
+  __syncwarp();
+  const int bit = 4 * bits * lane, wi = bit >> 5, sh = bit & 31;
+  atomicOr(stage + wi, field << sh);
+  if (sh + 4 * bits > 32) atomicOr(stage + wi + 1, field >> (32 - sh));
+  __syncwarp();
+  uint32_t* dst = reinterpret_cast<uint32_t*>(p.app_codes[side] + (tok * nb + blk) * 16 * bits);
+  if (lane < 4 * bits) dst[lane] = stage[lane];
+  if (lane == 0) {
+    __half nh = __float2half_rn(n);
+    if (__hisinf(nh)) {
+      nh = __ushort_as_half((unsigned short)0x7BFF);
+      if (p.status) atomicOr(p.status, TQ_DEV_NORM_OVERFLOW);
+    }
+    p.app_norms[side][tok * nb + blk] = __half_as_ushort(nh);
+  }
+}
+
 // How the flattened (unit, tile) space [0, T) is split over the persistent
 // CTAs.  Every unit's tiles cost 1 each and starting a unit costs kSwitchTiles
 // more (its query preparation, the drained copy ring, the partial's merge
@@ -540,6 +604,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   // parity) pairs, so V fragments come straight from the table.  GQ == 8:
   // one column per head, V fragments re-paired by token.
   static_assert(GQ == 4 || GQ == 8, "GQ");
+  static_assert(kCWarps >= 2 * NB, "the decode step appends one block per warp");
   constexpr bool kDup = GQ == 4;
   constexpr int kMT = kDup ? 4 : 8;  // V accumulator tiles per 128-block
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -874,6 +939,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     const int vlane = VB == 4 ? 8 * R : (VB == 3 ? 4 * ((3 * R) >> 1) : 4 * R);
     const uint32_t koff = (uint32_t)((2 * R) * NB * KBB + g * KB * 4);
     const uint32_t voff = (uint32_t)(SM::kOffSlotV + (4 * g) * NB * VBB + vlane);
+    // ---- decode step: the CTA that holds a unit's last tile first writes the
+    // sequence's new token (position len - 1) into the cache, K and V, one
+    // warp per 128-block, so that its own copies read it.  Other head groups
+    // of the same kv-head write the same bytes.
+    if (MODE != kSparseV && p.kv_new[0] != nullptr && seg_hi == nt && len > 0) {
+      if (cw < 2 * NB) {
+        append_block(p, cw / NB, cw % NB, (size_t)b * p.kv_heads + sg.kvh, cache_row + (len - 1), lane,
+                     reinterpret_cast<uint32_t*>(res) + 16 * cw);
+      }
+      __threadfence();
+      consumer_sync();
+    }
     // Warp cw takes tiles seg_lo + cw, seg_lo + cw + kCWarps, ...: tile i of
     // the warp (i = 0, 1, ...) lives in slot i % kDepth.  The first kDepth
     // copies are issued before the query preparation, which they overlap.

@@ -122,6 +122,102 @@ DecodeWorkspace decode_workspace_layout(int batch, int kv_heads, int q_heads, in
 
 }  // namespace tq
 
+namespace {
+
+// New-token rows of a decode step (null for plain decode attention).
+struct StepRows {
+  const void* k_new;
+  const void* v_new;
+  int kv_dtype;
+  uint8_t* k_codes;
+  uint16_t* k_norms;
+  uint8_t* v_codes;
+  uint16_t* v_norms;
+};
+
+int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                  int q_heads, const void* q, int q_dtype,
+                  const uint8_t* k_codes, const uint16_t* k_norms,
+                  const uint8_t* v_codes, const uint16_t* v_norms,
+                  const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                  void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                  void* stream, const StepRows* step) {
+  int st = check_desc(desc);
+  if (st != TQ_OK) return st;
+  if (desc->batch > tq::kMaxBatch || desc->head_dim > tq::kMaxDecodeHeadDim) return TQ_ERR_UNSUPPORTED;
+  if (desc->seq_cap % 2 != 0) return TQ_ERR_UNSUPPORTED;  // norm rows must start 4-byte aligned
+  if ((long long)desc->batch * ((desc->seq_cap + tq::kTile - 1) / tq::kTile) >= (1LL << 31))
+    return TQ_ERR_UNSUPPORTED;
+  if (q_heads < desc->kv_heads || q_heads % desc->kv_heads != 0) return TQ_ERR_INVALID_ARG;
+  if (q_dtype != TQ_F32 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+  if (!q || !k_codes || !k_norms || !v_codes || !v_norms || !seq_lens || !out)
+    return TQ_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_codes, 16) || !aligned(v_codes, 16) || !aligned(k_norms, 4) ||
+      !aligned(v_norms, 4) || !aligned(seq_lens, 4) || !aligned(out, 16))
+    return TQ_ERR_INVALID_ARG;
+  if (dev_status && !aligned(dev_status, 4)) return TQ_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || std::isnan(sparse_thr)) return TQ_ERR_INVALID_ARG;
+  if ((st = check_codebook(k_cb, desc->k_bits)) != TQ_OK) return st;
+  if ((st = check_codebook(v_cb, desc->v_bits)) != TQ_OK) return st;
+  if (step) {
+    if (step->kv_dtype != TQ_F32 && step->kv_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+    if (!step->k_new || !step->v_new || !aligned(step->k_new, 16) || !aligned(step->v_new, 16))
+      return TQ_ERR_INVALID_ARG;
+  }
+  const bool sparse = sparse_thr > 0.0f;
+  tq::DecodeWorkspace w = tq::decode_workspace_layout(desc->batch, desc->kv_heads, q_heads,
+                                                      desc->head_dim, desc->seq_cap, sparse);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return TQ_ERR_WORKSPACE;
+
+  tq::DecodeParams p{};
+  p.q = q;
+  p.q_f16 = q_dtype == TQ_F16;
+  p.k_codes = k_codes;
+  p.k_norms = k_norms;
+  p.v_codes = v_codes;
+  p.v_norms = v_norms;
+  p.seq_lens = seq_lens;
+  p.out = out;
+  p.status = dev_status;
+  char* base = static_cast<char*>(workspace);
+  p.tickets = reinterpret_cast<uint32_t*>(base + w.tickets_off);
+  p.slot_ml = reinterpret_cast<float*>(base + w.ml_off);
+  p.slot_acc = reinterpret_cast<float*>(base + w.acc_off);
+  p.scores = sparse ? reinterpret_cast<float*>(base + w.scores_off) : nullptr;
+  for (int j = 0; j < 16; ++j) {
+    p.kcent[j] = j < (1 << desc->k_bits) ? k_cb->centroids[j] : 0.0f;
+    p.vcent[j] = j < (1 << desc->v_bits) ? v_cb->centroids[j] : 0.0f;
+  }
+  sign_mask(desc->sign_seed, p.sign_mask);
+  p.k_bits = desc->k_bits;
+  p.v_bits = desc->v_bits;
+  p.batch = desc->batch;
+  p.kv_heads = desc->kv_heads;
+  p.q_heads = q_heads;
+  p.head_dim = desc->head_dim;
+  p.seq_cap = desc->seq_cap;
+  p.score_mult = (float)((double)scale * 1.4426950408889634 / tq::kBlock);
+  p.sparse_thr = sparse ? sparse_thr : 0.0f;
+  if (step) {
+    p.kv_new[0] = step->k_new;
+    p.kv_new[1] = step->v_new;
+    p.kv_new_f16 = step->kv_dtype == TQ_F16;
+    p.app_codes[0] = step->k_codes;
+    p.app_codes[1] = step->v_codes;
+    p.app_norms[0] = step->k_norms;
+    p.app_norms[1] = step->v_norms;
+    const tq_codebook* cbs[2] = {k_cb, v_cb};
+    const int bits[2] = {desc->k_bits, desc->v_bits};
+    for (int sd = 0; sd < 2; ++sd) {
+      const int levels = 1 << bits[sd];
+      for (int j = 0; j < levels / 2 - 1; ++j) p.pos_bounds[sd][j] = cbs[sd]->boundaries[levels / 2 + j];
+    }
+  }
+  return tq::launch_decode(p, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
 extern "C" {
 
 int tq_make_codebook(int bits, tq_codebook* out) {
@@ -219,58 +315,21 @@ int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const t
                         const int32_t* seq_lens, float scale, float sparse_thr, float* out,
                         void* workspace, size_t workspace_bytes, uint32_t* dev_status,
                         void* stream) {
-  int st = check_desc(desc);
-  if (st != TQ_OK) return st;
-  if (desc->batch > tq::kMaxBatch || desc->head_dim > tq::kMaxDecodeHeadDim) return TQ_ERR_UNSUPPORTED;
-  if (desc->seq_cap % 2 != 0) return TQ_ERR_UNSUPPORTED;  // norm rows must start 4-byte aligned
-  if ((long long)desc->batch * ((desc->seq_cap + tq::kTile - 1) / tq::kTile) >= (1LL << 31))
-    return TQ_ERR_UNSUPPORTED;
-  if (q_heads < desc->kv_heads || q_heads % desc->kv_heads != 0) return TQ_ERR_INVALID_ARG;
-  if (q_dtype != TQ_F32 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
-  if (!q || !k_codes || !k_norms || !v_codes || !v_norms || !seq_lens || !out)
-    return TQ_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k_codes, 16) || !aligned(v_codes, 16) || !aligned(k_norms, 4) ||
-      !aligned(v_norms, 4) || !aligned(seq_lens, 4) || !aligned(out, 16))
-    return TQ_ERR_INVALID_ARG;
-  if (dev_status && !aligned(dev_status, 4)) return TQ_ERR_INVALID_ARG;
-  if (!std::isfinite(scale) || std::isnan(sparse_thr)) return TQ_ERR_INVALID_ARG;
-  if ((st = check_codebook(k_cb, desc->k_bits)) != TQ_OK) return st;
-  if ((st = check_codebook(v_cb, desc->v_bits)) != TQ_OK) return st;
-  const bool sparse = sparse_thr > 0.0f;
-  tq::DecodeWorkspace w = tq::decode_workspace_layout(desc->batch, desc->kv_heads, q_heads,
-                                                      desc->head_dim, desc->seq_cap, sparse);
-  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return TQ_ERR_WORKSPACE;
+  return decode_common(desc, k_cb, v_cb, q_heads, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       nullptr);
+}
 
-  tq::DecodeParams p{};
-  p.q = q;
-  p.q_f16 = q_dtype == TQ_F16;
-  p.k_codes = k_codes;
-  p.k_norms = k_norms;
-  p.v_codes = v_codes;
-  p.v_norms = v_norms;
-  p.seq_lens = seq_lens;
-  p.out = out;
-  p.status = dev_status;
-  char* base = static_cast<char*>(workspace);
-  p.tickets = reinterpret_cast<uint32_t*>(base + w.tickets_off);
-  p.slot_ml = reinterpret_cast<float*>(base + w.ml_off);
-  p.slot_acc = reinterpret_cast<float*>(base + w.acc_off);
-  p.scores = sparse ? reinterpret_cast<float*>(base + w.scores_off) : nullptr;
-  for (int j = 0; j < 16; ++j) {
-    p.kcent[j] = j < (1 << desc->k_bits) ? k_cb->centroids[j] : 0.0f;
-    p.vcent[j] = j < (1 << desc->v_bits) ? v_cb->centroids[j] : 0.0f;
-  }
-  sign_mask(desc->sign_seed, p.sign_mask);
-  p.k_bits = desc->k_bits;
-  p.v_bits = desc->v_bits;
-  p.batch = desc->batch;
-  p.kv_heads = desc->kv_heads;
-  p.q_heads = q_heads;
-  p.head_dim = desc->head_dim;
-  p.seq_cap = desc->seq_cap;
-  p.score_mult = (float)((double)scale * 1.4426950408889634 / tq::kBlock);
-  p.sparse_thr = sparse ? sparse_thr : 0.0f;
-  return tq::launch_decode(p, static_cast<cudaStream_t>(stream));
+int tq_decode_step(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                   int q_heads, const void* q, int q_dtype, const void* k_new, const void* v_new,
+                   int kv_dtype, uint8_t* k_codes, uint16_t* k_norms, uint8_t* v_codes,
+                   uint16_t* v_norms, const int32_t* seq_lens, float scale, float sparse_thr,
+                   float* out, void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                   void* stream) {
+  const StepRows step{k_new, v_new, kv_dtype, k_codes, k_norms, v_codes, v_norms};
+  return decode_common(desc, k_cb, v_cb, q_heads, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       &step);
 }
 
 const char* tq_status_string(int status) {

@@ -54,6 +54,14 @@ struct DecodeParams {
   int batch, kv_heads, q_heads, head_dim, seq_cap;
   float score_mult;    // scale * log2(e) / 128
   float sparse_thr;    // > 0: two-pass exact sparse-V
+  // Decode step only (kv_new[0] != null): the new token of sequence b,
+  // rows [B, Hkv, D] of K and V, is encoded into the cache at position
+  // seq_lens[b] - 1 before attention reads it.
+  const void* kv_new[2];
+  int kv_new_f16;
+  uint8_t* app_codes[2];
+  uint16_t* app_norms[2];
+  float pos_bounds[2][7];  // positive decision boundaries of K and V, ascending
 };
 
 // Workspace layout shared by the size query and the launcher.

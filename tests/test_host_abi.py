@@ -24,7 +24,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol():
     names = _header_functions()
-    assert len(names) == 7
+    assert len(names) == 8
     lib = tq.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -138,6 +138,27 @@ def test_decode_rejects_bad_arguments_without_launch():
     assert lib.tq_decode_attention(ctypes.byref(odd), ctypes.byref(cb3), ctypes.byref(cb2), 8, _fake(GOOD), 1,
                                    _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), 0.1, 0.0,
                                    _fake(GOOD), _fake(GOOD), 1 << 30, None, None) == _lib.TQ_ERR_UNSUPPORTED
+
+
+def test_decode_step_rejects_bad_arguments_without_launch():
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+    need = tq.decode_workspace_size(d, 8)
+
+    def call(kn=GOOD, vn=GOOD, kvd=1, q=GOOD, wsb=None):
+        return lib.tq_decode_step(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), 8,
+                                  _fake(q) if q else None, 1, _fake(kn) if kn else None,
+                                  _fake(vn) if vn else None, kvd, _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                  _fake(GOOD), _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD),
+                                  need if wsb is None else wsb, None, None)
+
+    assert call(kn=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(vn=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(kn=GOOD + 8) == _lib.TQ_ERR_INVALID_ARG      # misaligned new rows
+    assert call(kvd=5) == _lib.TQ_ERR_INVALID_ARG
+    assert call(q=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(wsb=need - 1) == _lib.TQ_ERR_WORKSPACE
 
 
 def test_workspace_size_formula():
