@@ -8,9 +8,10 @@
 //
 // Kernel design (sm_100a):
 //  * Work = (unit, 16-token tile), unit = (batch, kv-head, group of <= 8
-//    q-heads).  All tiles of all units are laid end to end and cut into
-//    gridDim.x equal ranges, one per persistent CTA (stream-K style), so
-//    ragged lengths balance to within one tile.  A CTA writes one partial
+//    q-heads).  All tiles of all units are laid end to end and cut into one
+//    range per persistent CTA, one 16-warp CTA per SM.  The cut weighs each
+//    tile 1 and each unit start kSwitchTiles more, so CTAs whose range spans
+//    two units get fewer tiles (see Split).  A CTA writes one partial
 //    (m, l, acc) per unit it touches; the CTA that completes a unit (atomic
 //    tile count) merges the partials in a fixed order and applies the inverse
 //    rotation, so results do not depend on scheduling.
@@ -19,7 +20,7 @@
 //    (zero-filled past the end of the sequence) and waits for them with
 //    cp.async.wait_group, so several tiles per warp are in flight without
 //    holding registers, and no warp waits on another.
-//  * Scores: S[16 tok x 8 heads] = Kc[16 x 128] . Qhat[128 x 8] with
+//  * Scores: S[16 tok x 8 cols] = Kc[16 x 128] . Qhat[128 x 8] with
 //    mma.sync m16n8k16 (f16 in, f32 accumulate).  K codes are turned into f16
 //    A fragments in registers through a shared-memory table indexed by two
 //    codes and replicated per lane (conflict-free).  Contraction order is
@@ -27,12 +28,17 @@
 //  * Online softmax in the log2 domain with a lazy rescale (only when the
 //    running max grows by more than 2^6), exact because the stored max is the
 //    one every exponent used.
-//  * P.V: O^T[128 dims x 8 heads] += Vc^T[dims x 16 tok] . P'^T[16 tok x 8],
-//    P' = p * nV / 128; the score accumulator becomes the B fragment with two
+//  * P.V with up to four q-heads per kv-head (GQ = 4): the 8 MMA columns are
+//    (head, dim parity) pairs, so each V A-fragment register is one token's
+//    pair of adjacent dims straight from the table.  With more heads (GQ = 8)
+//    O^T[128 dims x 8 heads] += Vc^T[dims x 16 tok] . P'^T[16 tok x 8] with V
+//    re-paired by token.  P' = p * nV / 128 reaches the B fragment through two
 //    movmatrix transposes.  V stays in the rotated domain until the end.
 //  * Sparse-V is exact and two-pass: pass 1 stores log2-domain scores and
 //    per-partial (m, l); pass 2 forms the log-sum-exp, zeroes the normalised
 //    weights below the threshold and accumulates V with the rest.
+//  * Decode step: given the new token's K/V rows, the CTA holding a unit's
+//    last tile first encodes them into the cache (append_block).
 
 #include <cuda_fp16.h>
 
