@@ -197,9 +197,19 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
   for (int i = 0; i < 64; ++i) {
     const float y = (i & 1) ? x[i >> 1].y : x[i >> 1].x;
     const float a = fabsf(y);
-    int m = 0;
-#pragma unroll
-    for (int k = 0; k < NPOS; ++k) m += (a > thr[k]) ? 1 : 0;
+    // m = #{k : T_k < |y|/n}, found by bisection of the ascending T_k
+    int m;
+    if constexpr (NPOS == 1) {
+      m = (a > thr[0]) ? 1 : 0;
+    } else if constexpr (NPOS == 3) {
+      const int c1 = (a > thr[1]) ? 1 : 0;
+      m = 2 * c1 + ((a > (c1 ? thr[2] : thr[0])) ? 1 : 0);
+    } else {
+      const int c2 = (a > thr[3]) ? 1 : 0;
+      const int c1 = (a > (c2 ? thr[5] : thr[1])) ? 1 : 0;
+      const float t0 = c2 ? (c1 ? thr[6] : thr[4]) : (c1 ? thr[2] : thr[0]);
+      m = 4 * c2 + 2 * c1 + ((a > t0) ? 1 : 0);
+    }
     const int lowside = L / 2 - 1 - m;
     const uint32_t idx = (uint32_t)(y > 0.0f ? (lowside ^ (L - 1)) : lowside);
     g[i >> 3] |= idx << (BITS * (i & 7));
