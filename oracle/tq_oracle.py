@@ -361,6 +361,47 @@ def decode_rotated(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale,
     return out
 
 
+def attention_multi(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_lens, scale: float,
+                    sparse_thr: float = 0.0) -> np.ndarray:
+    """Multi-token queries in fp64 on dense K/V (the CUDA backend's
+    "multi-token" path of the [tq+ README] backend table; the pages give no
+    detail, so: n_q query tokens per sequence are its last n_q positions, as in
+    a speculative or chunked decode step).
+
+    q: [B, n_q, Hq, D]; k, v: [B, Hkv, S, D].  Query token j of sequence b sits
+    at position p_j = seq_lens[b] - n_q + j and sees positions t <= p_j: the
+    scores form one [n, n_q] matrix with the causal mask t <= p_j applied
+    column by column, then softmax per column.  Sparse-V as in attention().
+    A token with p_j < 0 gives a zero row.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    bsz, n_q, hq, d = q.shape
+    group = hq // k.shape[1]
+    out = np.zeros((bsz, n_q, hq, d))
+    for b in range(bsz):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        t = np.arange(n)[:, None]
+        p = n - n_q + np.arange(n_q)[None, :]
+        visible = t <= p                                      # [n, n_q]
+        for h in range(hq):
+            kv = h // group
+            s = scale * (k[b, kv, :n] @ q[b, :, h].T)         # [n, n_q]
+            s = np.where(visible, s, -np.inf)
+            for j in range(n_q):
+                if p[0, j] < 0:
+                    continue
+                w = np.exp(s[:, j] - s[:, j].max())
+                w = w / w.sum()
+                if sparse_thr > 0:
+                    w = np.where(w < sparse_thr, 0.0, w)
+                out[b, j, h] = w @ v[b, kv, :n]
+    return out
+
+
 def sparse_skip_fraction(q, k, seq_lens, scale, thr, group):
     """Fraction of (q-head, position) pairs whose normalised weight is < thr."""
     q = np.asarray(q, dtype=np.float64)

@@ -313,3 +313,57 @@ def test_attention_weights_match_torch_softmax():
         n = [20, 7][b]
         ref = torch.softmax(torch.tensor(k[b, h // 2, :n] @ q[b, h]) * 0.1, dim=0).numpy()
         np.testing.assert_allclose(w, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_multi_token_attention_single_token_is_decode():
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((2, 8, 128))
+    k = rng.standard_normal((2, 2, 40, 128))
+    v = rng.standard_normal((2, 2, 40, 128))
+    lens = [40, 9]
+    got = O.attention_multi(q[:, None], k, v, lens, 0.09)[:, 0]
+    np.testing.assert_allclose(got, O.attention(q, k, v, lens, 0.09), rtol=1e-12, atol=1e-12)
+
+
+def test_multi_token_attention_matches_torch_sdpa_with_causal_mask():
+    """Query token j of a sequence of length n sits at n - n_q + j and sees
+    t <= n - n_q + j: an explicit boolean mask for torch's SDPA."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(22)
+    n_q, scale = 5, 1 / math.sqrt(128)
+    q = rng.standard_normal((2, n_q, 8, 128))
+    k = rng.standard_normal((2, 2, 30, 128))
+    v = rng.standard_normal((2, 2, 30, 128))
+    lens = [30, 12]
+    ours = O.attention_multi(q, k, v, lens, scale)
+    for b in range(2):
+        n = lens[b]
+        qt = torch.tensor(q[b].transpose(1, 0, 2))                  # [Hq, n_q, D]
+        kt = torch.tensor(np.repeat(k[b, :, :n], 4, axis=0))       # [Hq, n, D]
+        vt = torch.tensor(np.repeat(v[b, :, :n], 4, axis=0))
+        mask = torch.tensor(np.arange(n)[None, :] <= (n - n_q + np.arange(n_q))[:, None])  # [n_q, n]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(ours[b], ref.numpy().transpose(1, 0, 2), rtol=1e-12, atol=1e-12)
+
+
+def test_multi_token_attention_is_decode_at_each_position():
+    """Token j equals single-token attention over the first n - n_q + j + 1
+    positions; a token before the sequence start gives zeros; positions past
+    seq_lens never matter."""
+    rng = np.random.default_rng(23)
+    n_q = 4
+    q = rng.standard_normal((3, n_q, 4, 128))
+    k = rng.standard_normal((3, 1, 20, 128))
+    v = rng.standard_normal((3, 1, 20, 128))
+    lens = np.array([20, 7, 2])
+    got = O.attention_multi(q, k, v, lens, 0.1, sparse_thr=1e-3)
+    for j in range(n_q):
+        lj = np.maximum(lens - n_q + j + 1, 0)
+        want = O.attention(q[:, j], k, v, lj, 0.1, sparse_thr=1e-3)
+        np.testing.assert_allclose(got[:, j], want, rtol=1e-12, atol=1e-12)
+    assert np.all(got[2, :2] == 0.0)                                # positions -2, -1
+    k2, v2 = k.copy(), v.copy()
+    k2[1, :, 7:] = 1e6
+    v2[1, :, 7:] = np.nan
+    np.testing.assert_array_equal(O.attention_multi(q, k2, v2, lens, 0.1)[1],
+                                  O.attention_multi(q, k, v, lens, 0.1)[1])
