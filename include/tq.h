@@ -177,6 +177,33 @@ int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const t
                         void* stream);
 
 /*
+ * tq_decode_attention_multi -- n_q query tokens per sequence (a speculative
+ * or chunked decode step) against the packed cache.  The README backend table
+ * lists CUDA "multi-token" paths without detail; here the n_q tokens are the
+ * last n_q positions of each sequence, and query token j (position
+ * seq_lens[b] - n_q + j) sees the positions up to its own:
+ *   out[b, j, h] = tq_decode_attention output of q[b, j, h] over positions
+ *                  [0, seq_lens[b] - n_q + j], zero when that range is empty.
+ * All n_q tokens of a sequence are computed from the same K/V fragments of
+ * each tile (the codes are turned into MMA operands once per tile).
+ *   - n_q: 1..TQ_MAX_QUERY_TOKENS.
+ *   - q: device [batch, n_q, q_heads, head_dim]; out: fp32 [batch, n_q,
+ *     q_heads, head_dim].
+ *   - workspace: tq_decode_workspace_size(desc, q_heads * n_q, sparse_thr)
+ *     bytes.
+ * Every other argument, limit and error is that of tq_decode_attention
+ * (n_q = 1 gives exactly its results).
+ */
+#define TQ_MAX_QUERY_TOKENS 16
+int tq_decode_attention_multi(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                              const tq_codebook* v_cb, int q_heads, int n_q, const void* q,
+                              int q_dtype, const uint8_t* k_codes, const uint16_t* k_norms,
+                              const uint8_t* v_codes, const uint16_t* v_norms,
+                              const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                              void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                              void* stream);
+
+/*
  * tq_decode_step -- one decode step in one launch: append every sequence's
  * new token to the cache, then attend over the cache including it.  In a
  * decode step the new token's K/V rows are written into the quantised cache

@@ -12,6 +12,7 @@ TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ
 TQ_NOALLOC_SCRATCH_BYTES = 64 << 20
 TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE = 1, 2, 4
 TQ_F32, TQ_F16 = 0, 1
+TQ_MAX_QUERY_TOKENS = 16
 
 # Every symbol include/tq.h declares, with (restype, argtypes).
 c_int, c_float, c_size_t, c_void_p = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
@@ -40,6 +41,9 @@ SIGNATURES = {
     "tq_decode_attention": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                                     c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "tq_decode_attention_multi": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_int, c_void_p,
+                                          c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
+                                          c_float, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "tq_decode_step": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
                                c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                c_void_p, c_float, c_float, c_void_p, c_void_p, c_size_t, c_void_p,

@@ -138,6 +138,24 @@ def decode_attention(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, 
     return out
 
 
+def decode_attention_multi(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, seq_lens, scale: float,
+                           out, workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """n_q query tokens per sequence, the last n_q positions, each seeing the
+    positions up to its own (tq_decode_attention_multi).  q, out: [B, n_q, Hq, D];
+    workspace: alloc_workspace(desc, Hq * n_q, sparse_thr)."""
+    n_q, q_heads = q.shape[1], q.shape[2]
+    st = lib().tq_decode_attention_multi(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb), q_heads, n_q,
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention_multi", st)
+    return out
+
+
 def decode_step(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, k_new, v_new, seq_lens, scale: float,
                 out, workspace, sparse_thr: float = 0.0, status=None, stream=None):
     """One decode step (tq_decode_step): write each sequence's new K/V row

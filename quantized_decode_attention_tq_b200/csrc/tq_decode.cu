@@ -589,7 +589,7 @@ __device__ __forceinline__ Segment locate(long long x, long long hi, const int* 
   s.unit = bl * UB + s.r;
   s.kvh = s.r / n_hg;
   s.hg = s.r % n_hg;
-  s.h0 = s.kvh * G + s.hg * kMaxGroup;
+  s.h0 = s.kvh * G + s.hg * kMaxGroup;  // first (virtual) head of the unit
   s.Gu = min(kMaxGroup, G - s.hg * kMaxGroup);
   s.len = min(max(__ldg(seq_lens + bl), 0), seq_cap);
   return s;
@@ -649,9 +649,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   // kDup B fragments: a token's weight in the low half (s' = 0, R < 4) or
   // the high half (s' = 1) of the register, zero in the other
   const uint32_t selLo = R < 4 ? 0x4410u : 0x1044u, selHi = R < 4 ? 0x4432u : 0x3244u;
+  // Heads of a unit are "virtual heads" (query token j, q-head h of the
+  // kv-head's group), vl = j * G + h, so n_q query tokens per sequence share
+  // the K/V fragments of each tile.  Virtual head vh = kvh * Gv + vl of batch
+  // entry b reads q and writes out row (b * n_q + j) * q_heads + kvh * G + h.
   const int G = p.q_heads / p.kv_heads;
-  const int n_hg = (G + kMaxGroup - 1) / kMaxGroup;
+  const int Gv = G * p.n_q;
+  const int n_hg = (Gv + kMaxGroup - 1) / kMaxGroup;
   const int UB = p.kv_heads * n_hg;  // units per batch entry
+  auto vrow = [&](int b, int vh) -> size_t {
+    const int kvh = vh / Gv, vl = vh % Gv;
+    return ((size_t)b * p.n_q + vl / G) * p.q_heads + kvh * G + vl % G;
+  };
 
   // ---- tables: code pair -> half2 codewords, replicated for every lane ----
   if constexpr (HASK) {
@@ -707,9 +716,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 
   // ---- zero rows of empty sequences (only the V-producing passes) ---------
   if constexpr (MODE != kScores) {
-    const long long rows = (long long)p.batch * p.q_heads;
+    const long long rows = (long long)p.batch * p.n_q * p.q_heads;
     for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
-      const int b = (int)(row / p.q_heads);
+      const int b = (int)(row / ((long long)p.n_q * p.q_heads));
       if (prefix[b + 1] == prefix[b]) {
         for (int d = tid; d < D; d += kThreads) p.out[row * D + d] = 0.0f;
       }
@@ -733,7 +742,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       float v[NB][4];
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
-        const size_t qi = ((size_t)b * p.q_heads + h0 + j) * D + blk * kBlock + 4 * lane;
+        const size_t qi = vrow(b, h0 + j) * D + blk * kBlock + 4 * lane;
         if (j >= Gu) {
           v[blk][0] = v[blk][1] = v[blk][2] = v[blk][3] = 0.0f;
         } else if (p.q_f16) {
@@ -802,10 +811,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       for (int blk = 0; blk < NB; ++blk) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          if constexpr (MODE == kFused) v[blk][k] = v[blk][k] / L;
+          if constexpr (MODE == kFused) v[blk][k] = L > 0.0f ? v[blk][k] / L : 0.0f;  // L = 0: no position seen
           if ((sgn >> k) & 1u) v[blk][k] = -v[blk][k];
         }
-        *reinterpret_cast<float4*>(p.out + ((size_t)b * p.q_heads + h0 + hd) * D + blk * kBlock + 4 * lane) =
+        *reinterpret_cast<float4*>(p.out + vrow(b, h0 + hd) * D + blk * kBlock + 4 * lane) =
             make_float4(v[blk][0], v[blk][1], v[blk][2], v[blk][3]);
       }
     }
@@ -884,7 +893,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   };
 
   for (long long x = lo; x < hi;) {
-    const Segment sg = locate(x, hi, prefix, p.batch, UB, n_hg, G, p.seq_cap, p.seq_lens);
+    const Segment sg = locate(x, hi, prefix, p.batch, UB, n_hg, Gv, p.seq_cap, p.seq_lens);
     const int b = sg.b, nt = sg.nt, unit = sg.unit, h0 = sg.h0, Gu = sg.Gu, len = sg.len;
     const int seg_lo = sg.seg_lo, seg_hi = sg.seg_hi;
     const long long Su = sg.Su;
@@ -1032,11 +1041,28 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 
     // Phase 2 of a tile: scale and mask the scores, online softmax (D4) or the
     // sparse-V gate (D5), then the V sum in the rotated domain (D6).
+    // Positions each of this lane's two score columns may see: query token j
+    // of the sequence sits at len - n_q + j and sees the positions up to its
+    // own.  Padding columns (head >= Gu) see the whole sequence.
+    int lim[2];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int hd = kDup ? (2 * g + cc) & 3 : 2 * g + cc;
+      const int tok = (sg.hg * kMaxGroup + hd) / G;
+      lim[cc] = hd < Gu ? min(len, len - p.n_q + tok + 1) : len;
+    }
+    const int len_full = len - p.n_q + 1;  // tiles ending here see no mask at all
+
     auto finish = [&](const TileRegs<KB, VB, NB>& tr, int tile, const Raw& raw, auto full_tag) {
       constexpr bool FULL = decltype(full_tag)::value;
       const int t0 = tile * kTile;
       // rows R and R+8 of the score tile are tokens 2R and 2R+1
-      const bool okR = FULL || t0 + 2 * R < len, okR8 = FULL || t0 + 2 * R + 1 < len;
+      bool okR[2], okR8[2];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        okR[cc] = FULL || t0 + 2 * R < lim[cc];
+        okR8[cc] = FULL || t0 + 2 * R + 1 < lim[cc];
+      }
       float pR[2], pR8[2];
       if constexpr (HASK) {
         float sR[2], sR8[2];
@@ -1049,18 +1075,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             a = fmaf(raw.c[blk][cc], kn.x, a);
             bb = fmaf(raw.c[blk][2 + cc], kn.y, bb);
           }
-          sR[cc] = okR ? a * qmul[cc] : -INFINITY;
-          sR8[cc] = okR8 ? bb * qmul[cc] : -INFINITY;
+          sR[cc] = okR[cc] ? a * qmul[cc] : -INFINITY;
+          sR8[cc] = okR8[cc] ? bb * qmul[cc] : -INFINITY;
         }
         if constexpr (MODE == kScores) {
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             const int hd = 2 * g + cc;  // columns 4..7 repeat heads 0..3 when kDup
             if (hd < Gu && (!kDup || g < 2)) {
-              float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap + t0 + 2 * R;
-              if (okR8) {
+              float* srow = p.scores + ((size_t)b * p.kv_heads * Gv + h0 + hd) * p.seq_cap + t0 + 2 * R;
+              if (okR8[cc]) {
                 *reinterpret_cast<float2*>(srow) = make_float2(sR[cc], sR8[cc]);
-              } else if (okR) {
+              } else if (okR[cc]) {
                 srow[0] = sR[cc];
               }
             }
@@ -1095,8 +1121,11 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         }
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          pR[cc] = ex2(sR[cc] - m_run[cc]);
-          pR8[cc] = ex2(sR8[cc] - m_run[cc]);
+          // a column that has seen no position yet (a later query token's
+          // causal limit) keeps m = -inf: its weights are 0, not NaN
+          const float mref = m_run[cc] == -INFINITY ? 0.0f : m_run[cc];
+          pR[cc] = ex2(sR[cc] - mref);
+          pR8[cc] = ex2(sR8[cc] - mref);
           l_run[cc] += pR[cc] + pR8[cc];
         }
       } else {
@@ -1106,13 +1135,13 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           const int hd = kDup ? (2 * g + cc) & 3 : 2 * g + cc;
           float wR = 0.0f, wR8 = 0.0f;
           if (hd < Gu) {
-            const float* srow = p.scores + ((size_t)b * p.q_heads + h0 + hd) * p.seq_cap + t0 + 2 * R;
+            const float* srow = p.scores + ((size_t)b * p.kv_heads * Gv + h0 + hd) * p.seq_cap + t0 + 2 * R;
             float s0 = -INFINITY, s1 = -INFINITY;
-            if (okR8) {
+            if (okR8[cc]) {
               const float2 sv = __ldcs(reinterpret_cast<const float2*>(srow));
               s0 = sv.x;
               s1 = sv.y;
-            } else if (okR) {
+            } else if (okR[cc]) {
               s0 = __ldcs(srow);
             }
             const float d0 = s0 - lse2[cc], d1 = s1 - lse2[cc];
@@ -1189,7 +1218,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         cp_async_commit();
         const int tile = first + i * kCWarps;
         const Raw raw = scores(tr);
-        if (tile * kTile + kTile <= len)
+        if (tile * kTile + kTile <= len_full)
           finish(tr, tile, raw, std::true_type{});
         else
           finish(tr, tile, raw, std::false_type{});
@@ -1350,7 +1379,7 @@ int dispatch_modes(const DecodeParams& p, cudaStream_t stream) {
 
 template <int KB, int VB, int NB>
 int dispatch_gq(const DecodeParams& p, cudaStream_t stream) {
-  if (p.q_heads / p.kv_heads <= 4) return dispatch_modes<KB, VB, NB, 4>(p, stream);
+  if (p.q_heads / p.kv_heads * p.n_q <= 4) return dispatch_modes<KB, VB, NB, 4>(p, stream);
   return dispatch_modes<KB, VB, NB, 8>(p, stream);
 }
 

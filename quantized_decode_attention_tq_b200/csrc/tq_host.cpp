@@ -136,7 +136,7 @@ struct StepRows {
 };
 
 int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
-                  int q_heads, const void* q, int q_dtype,
+                  int q_heads, int n_q, const void* q, int q_dtype,
                   const uint8_t* k_codes, const uint16_t* k_norms,
                   const uint8_t* v_codes, const uint16_t* v_norms,
                   const int32_t* seq_lens, float scale, float sparse_thr, float* out,
@@ -149,6 +149,7 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
   if ((long long)desc->batch * ((desc->seq_cap + tq::kTile - 1) / tq::kTile) >= (1LL << 31))
     return TQ_ERR_UNSUPPORTED;
   if (q_heads < desc->kv_heads || q_heads % desc->kv_heads != 0) return TQ_ERR_INVALID_ARG;
+  if (n_q < 1 || n_q > TQ_MAX_QUERY_TOKENS) return TQ_ERR_INVALID_ARG;
   if (q_dtype != TQ_F32 && q_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
   if (!q || !k_codes || !k_norms || !v_codes || !v_norms || !seq_lens || !out)
     return TQ_ERR_INVALID_ARG;
@@ -165,7 +166,7 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
       return TQ_ERR_INVALID_ARG;
   }
   const bool sparse = sparse_thr > 0.0f;
-  tq::DecodeWorkspace w = tq::decode_workspace_layout(desc->batch, desc->kv_heads, q_heads,
+  tq::DecodeWorkspace w = tq::decode_workspace_layout(desc->batch, desc->kv_heads, q_heads * n_q,
                                                       desc->head_dim, desc->seq_cap, sparse);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.total) return TQ_ERR_WORKSPACE;
 
@@ -198,6 +199,7 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
   p.seq_cap = desc->seq_cap;
   p.score_mult = (float)((double)scale * 1.4426950408889634 / tq::kBlock);
   p.sparse_thr = sparse ? sparse_thr : 0.0f;
+  p.n_q = n_q;
   if (step) {
     p.kv_new[0] = step->k_new;
     p.kv_new[1] = step->v_new;
@@ -315,7 +317,19 @@ int tq_decode_attention(const tq_kv_desc* desc, const tq_codebook* k_cb, const t
                         const int32_t* seq_lens, float scale, float sparse_thr, float* out,
                         void* workspace, size_t workspace_bytes, uint32_t* dev_status,
                         void* stream) {
-  return decode_common(desc, k_cb, v_cb, q_heads, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+  return decode_common(desc, k_cb, v_cb, q_heads, 1, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       nullptr);
+}
+
+int tq_decode_attention_multi(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                              const tq_codebook* v_cb, int q_heads, int n_q, const void* q,
+                              int q_dtype, const uint8_t* k_codes, const uint16_t* k_norms,
+                              const uint8_t* v_codes, const uint16_t* v_norms,
+                              const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                              void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                              void* stream) {
+  return decode_common(desc, k_cb, v_cb, q_heads, n_q, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
                        seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
                        nullptr);
 }
@@ -327,7 +341,7 @@ int tq_decode_step(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_cod
                    float* out, void* workspace, size_t workspace_bytes, uint32_t* dev_status,
                    void* stream) {
   const StepRows step{k_new, v_new, kv_dtype, k_codes, k_norms, v_codes, v_norms};
-  return decode_common(desc, k_cb, v_cb, q_heads, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+  return decode_common(desc, k_cb, v_cb, q_heads, 1, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
                        seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
                        &step);
 }

@@ -54,6 +54,7 @@ struct DecodeParams {
   int batch, kv_heads, q_heads, head_dim, seq_cap;
   float score_mult;    // scale * log2(e) / 128
   float sparse_thr;    // > 0: two-pass exact sparse-V
+  int n_q;             // query tokens per sequence (the last n_q positions, causal)
   // Decode step only (kv_new[0] != null): the new token of sequence b,
   // rows [B, Hkv, D] of K and V, is encoded into the cache at position
   // seq_lens[b] - 1 before attention reads it.

@@ -24,7 +24,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol():
     names = _header_functions()
-    assert len(names) == 8
+    assert len(names) == 9
     lib = tq.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -159,6 +159,27 @@ def test_decode_step_rejects_bad_arguments_without_launch():
     assert call(kvd=5) == _lib.TQ_ERR_INVALID_ARG
     assert call(q=0) == _lib.TQ_ERR_INVALID_ARG
     assert call(wsb=need - 1) == _lib.TQ_ERR_WORKSPACE
+
+
+def test_decode_multi_rejects_bad_token_counts():
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+
+    def call(n_q):
+        need = tq.decode_workspace_size(d, 8 * max(n_q, 1))
+        return lib.tq_decode_attention_multi(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), 8, n_q,
+                                             _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                             _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD), need, None, None)
+
+    assert call(0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(_lib.TQ_MAX_QUERY_TOKENS + 1) == _lib.TQ_ERR_INVALID_ARG
+    # the workspace must be sized for q_heads * n_q
+    need1 = tq.decode_workspace_size(d, 8)
+    assert lib.tq_decode_attention_multi(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), 8, 4,
+                                         _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                         _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD), need1, None,
+                                         None) == _lib.TQ_ERR_WORKSPACE
 
 
 def test_workspace_size_formula():
