@@ -55,6 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
     ap.add_argument("--workload", choices=sorted(WORKLOAD_NAMES), default="gqa")
     ap.add_argument("--no-encode", action="store_true", help="skip the encode-only measurement")
+    ap.add_argument("--no-multi", action="store_true", help="skip the multi-token measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -374,6 +375,35 @@ def run_tq(args):
     e2e_ms = allmax(e0.elapsed_time(e1) / args.steps)
     e2e_value = tokens_step / (e2e_ms / 1e3)
 
+    # ---- multi-token queries on the same caches (n_q causal query tokens) ---
+    multi_info = None
+    if rank == 0 and not args.no_multi:
+        try:
+            multi_info = {"workload": "the same caches and lengths; n_q query tokens per sequence "
+                                      "(its last n_q positions, causal)", "us_per_launch": {},
+                          "us_per_query_token": {}}
+            for n_q in (2, 4):
+                qm = torch.randn(w.batch, n_q, w.q_heads, w.head_dim, device=dev).to(q.dtype)
+                om = torch.empty(w.batch, n_q, w.q_heads, w.head_dim, dtype=torch.float32, device=dev)
+                wsm = tq.alloc_workspace(desc, w.q_heads * n_q, w.sparse_thr, dev)
+                for i in range(3):
+                    tq.decode_attention_multi(caches[i % n_copies], kcb, vcb, qm, lens, w.scale, om, wsm,
+                                              sparse_thr=w.sparse_thr)
+                m0 = torch.cuda.Event(enable_timing=True)
+                m1 = torch.cuda.Event(enable_timing=True)
+                m0.record(stream)
+                for i in range(10):
+                    tq.decode_attention_multi(caches[i % n_copies], kcb, vcb, qm, lens, w.scale, om, wsm,
+                                              sparse_thr=w.sparse_thr)
+                m1.record(stream)
+                torch.cuda.synchronize()
+                us = m0.elapsed_time(m1) / 10 * 1e3
+                multi_info["us_per_launch"][str(n_q)] = us
+                multi_info["us_per_query_token"][str(n_q)] = us / n_q
+                del qm, om, wsm
+        except Exception as e:  # reported, never fatal to the benchmark line
+            multi_info = {"error": f"{type(e).__name__}: {e}"}
+
     # ---- encoder alone on the encode-only workload -------------------------
     encode_info = None
     if not args.no_encode and rank == 0:
@@ -442,6 +472,7 @@ def run_tq(args):
             "gpu_launches": args.steps * decode_launches,
             "clocks": clocks,
             "encode": encode_info,
+            "multi_token": multi_info,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
