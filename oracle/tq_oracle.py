@@ -24,7 +24,7 @@ Pages cited (by title and section):
                   §3.3 "Lloyd-Max量化算法" (init centres, assign to nearest,
                   centre = mean of its points, repeat), §4.1 table (bits/ratio).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * rotation order H.D (signs first, then the unnormalised Sylvester WHT);
   * sign vector from SplitMix64 (Steele, Lea, Flood 2014), state = seed,
     s_i = -1 when the top bit of the i-th output is set;

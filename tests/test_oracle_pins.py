@@ -367,3 +367,133 @@ def test_multi_token_attention_is_decode_at_each_position():
     v2[1, :, 7:] = np.nan
     np.testing.assert_array_equal(O.attention_multi(q, k2, v2, lens, 0.1)[1],
                                   O.attention_multi(q, k, v, lens, 0.1)[1])
+
+
+# --------------------------------------------------------- sparse-V gate ---
+# README "压缩策略" and "TurboQuant+" section "注意力门控稀疏V解压": V rows whose
+# softmax weight is below the threshold are skipped and count as zero.  The
+# weight is the normalised softmax weight; the kept weights are not rescaled.
+# The reference below is torch.softmax (a library routine) with the mask
+# applied to its output, so neither slip of the oracle's gate -- gating on the
+# unnormalised exp(s - max), or renormalising the kept weights -- can hide.
+
+
+def _torch_gated(q, k, v, lens, scale, thr, limits=None):
+    """o[b, h] = sum_t [w_t >= thr] w_t v_t with w = torch.softmax(scale q.k)."""
+    torch = pytest.importorskip("torch")
+    group = q.shape[1] // k.shape[1]
+    out = np.zeros(q.shape)
+    for b in range(q.shape[0]):
+        n = int(lens[b] if limits is None else limits[b])
+        if n <= 0:
+            continue
+        for h in range(q.shape[1]):
+            kv = h // group
+            s = torch.tensor(k[b, kv, :n] @ q[b, h], dtype=torch.float64) * scale
+            w = torch.softmax(s, dim=0)
+            w = torch.where(w >= thr, w, torch.zeros_like(w))
+            out[b, h] = (w @ torch.tensor(v[b, kv, :n], dtype=torch.float64)).numpy()
+    return out
+
+
+def _slips(q, k, v, lens, scale, thr):
+    """The two plausible wrong gates, for checking that a case discriminates."""
+    group = q.shape[1] // k.shape[1]
+    unnorm = np.zeros(q.shape)
+    renorm = np.zeros(q.shape)
+    for b in range(q.shape[0]):
+        n = int(lens[b])
+        for h in range(q.shape[1]):
+            kv = h // group
+            s = scale * (k[b, kv, :n] @ q[b, h])
+            e = np.exp(s - s.max())
+            w = e / e.sum()
+            keep_u = e >= thr
+            unnorm[b, h] = (w * keep_u) @ v[b, kv, :n]
+            keep = w >= thr
+            renorm[b, h] = (w * keep / max((w * keep).sum(), 1e-300)) @ v[b, kv, :n]
+    return unnorm, renorm
+
+
+def _gate_case(rng, bsz=2, hkv=2, group=3, n=160, d=128):
+    q = rng.standard_normal((bsz, hkv * group, d)) * 1.5
+    k = rng.standard_normal((bsz, hkv, n, d))
+    v = rng.standard_normal((bsz, hkv, n, d))
+    return q, k, v
+
+
+def test_sparse_gate_dense_attention_matches_masked_torch_softmax():
+    rng = np.random.default_rng(31)
+    q, k, v = _gate_case(rng)
+    lens = [160, 97]
+    scale = 1 / math.sqrt(128)
+    for thr in (0.5 / 160, 1.0 / 160, 3e-3):
+        ref = _torch_gated(q, k, v, lens, scale, thr)
+        np.testing.assert_allclose(O.attention(q, k, v, lens, scale, thr), ref, rtol=0, atol=1e-12)
+        # the case discriminates: both slips move the output by far more
+        unnorm, renorm = _slips(q, k, v, lens, scale, thr)
+        assert np.max(np.abs(unnorm - ref)) > 1e-2 and np.max(np.abs(renorm - ref)) > 1e-2
+
+
+def test_sparse_gate_of_both_cache_formulations_matches_masked_torch_softmax():
+    rng = np.random.default_rng(32)
+    s, (ck, cv), _, (kc, kn, vc, vn) = _random_cache(rng, 2, 2, 120, 256, 3, 2)
+    kt = O.dequantize(kc, kn, 3, ck, s)
+    vt = O.dequantize(vc, vn, 2, cv, s)
+    q = rng.standard_normal((2, 6, 256)) * 1.5
+    lens = [120, 45]
+    scale = 1 / 16
+    # thresholds at the median and the upper quartile of the weights drop a
+    # large share of the mass
+    w_all = np.concatenate([w for w in O.attention_weights(q, kt, lens, scale).values()])
+    for thr in (np.quantile(w_all, 0.5), np.quantile(w_all, 0.75), 1.0 / 120):
+        ref = _torch_gated(q, kt, vt, lens, scale, thr)
+        a = O.decode_dequant(q, kc, kn, vc, vn, lens, scale, 3, 2, ck, cv, s, thr)
+        b = O.decode_rotated(q, kc, kn, vc, vn, lens, scale, 3, 2, ck, cv, s, thr)
+        tol = 1e-10 * np.max(np.abs(ref))
+        assert np.max(np.abs(a - ref)) <= tol and np.max(np.abs(b - ref)) <= tol
+        unnorm, renorm = _slips(q, kt, vt, lens, scale, thr)
+        assert np.max(np.abs(unnorm - ref)) > 1e-2 * np.max(np.abs(ref))
+        assert np.max(np.abs(renorm - ref)) > 1e-2 * np.max(np.abs(ref))
+
+
+def test_sparse_gate_of_multi_token_attention_matches_masked_torch_softmax():
+    """Query token j sees positions t <= n - n_q + j; its gate uses the
+    softmax over exactly those positions."""
+    rng = np.random.default_rng(33)
+    n_q = 3
+    q = rng.standard_normal((2, n_q, 4, 128)) * 1.5
+    k = rng.standard_normal((2, 2, 90, 128))
+    v = rng.standard_normal((2, 2, 90, 128))
+    lens = np.array([90, 40])
+    scale = 1 / math.sqrt(128)
+    for thr in (0.5 / 90, 1.0 / 60):
+        got = O.attention_multi(q, k, v, lens, scale, thr)
+        for j in range(n_q):
+            lim = lens - n_q + j + 1
+            ref = _torch_gated(q[:, j], k, v, lens, scale, thr, limits=lim)
+            np.testing.assert_allclose(got[:, j], ref, rtol=0, atol=1e-12)
+            unnorm, renorm = _slips(q[:, j], k, v, lim, scale, thr)
+            assert np.max(np.abs(unnorm - ref)) > 1e-2 and np.max(np.abs(renorm - ref)) > 1e-2
+
+
+def test_sparse_gate_keeps_weights_at_the_threshold_and_drops_below():
+    """Hand-built scores: n/2 positions at score 1 and n/2 at 0, so the
+    normalised weights are e/Z and 1/Z with Z = n/2 (e + 1).  A threshold
+    between them keeps only the first half, unrescaled: o = (e/Z) sum of
+    their V rows.  A threshold above both drops everything (an unnormalised
+    gate would keep every position there)."""
+    n, d = 40, 128
+    q = np.zeros((1, 1, d))
+    q[0, 0, 0] = 1.0
+    k = np.zeros((1, 1, n, d))
+    k[0, 0, : n // 2, 0] = 1.0
+    rng = np.random.default_rng(34)
+    v = rng.standard_normal((1, 1, n, d))
+    z = n / 2 * (math.e + 1)
+    hi, lo = math.e / z, 1 / z
+    kept = O.attention(q, k, v, [n], 1.0, sparse_thr=(hi + lo) / 2)
+    np.testing.assert_allclose(kept[0, 0], hi * v[0, 0, : n // 2].sum(axis=0), rtol=1e-12, atol=1e-13)
+    at = O.attention(q, k, v, [n], 1.0, sparse_thr=lo)      # w == thr is kept
+    np.testing.assert_allclose(at, O.attention(q, k, v, [n], 1.0), rtol=1e-12, atol=1e-13)
+    assert np.all(O.attention(q, k, v, [n], 1.0, sparse_thr=2 * hi) == 0.0)
