@@ -60,7 +60,8 @@ typedef enum {
   TQ_ERR_UNSUPPORTED = 2,  /* valid but not built: bits, head_dim, group     */
   TQ_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required     */
   TQ_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute) */
-  TQ_ERR_SCRATCH_LIMIT = 5 /* needs more than the built-in scratch array      */
+  TQ_ERR_DEVICE_BOUNDS = 5,/* tq_read_device_status: a range bit is set      */
+  TQ_ERR_SCRATCH_LIMIT = 6 /* needs more than the built-in scratch array      */
 } tq_status;
 
 /* Bits of the device status word (sticky; the library only ORs into it). */
@@ -213,9 +214,11 @@ int tq_decode_attention_multi(const tq_kv_desc* desc, const tq_codebook* k_cb,
  *   - seq_lens counts the new token: for sequence b, rows k_new[b, h, :] and
  *     v_new[b, h, :] are encoded exactly as tq_encode_kv would (block norm,
  *     signs, WHT, codebook index, packing) and written at position
- *     seq_lens[b] - 1, after seq_lens is clamped to [0, seq_cap]
- *     (TQ_DEV_LEN_RANGE); a sequence of length 0 appends nothing.  Then the
- *     output is that of tq_decode_attention over positions [0, seq_lens[b]).
+ *     seq_lens[b] - 1.  A sequence whose seq_lens[b] is outside [1, seq_cap]
+ *     appends nothing, so no cached token is overwritten (values outside
+ *     [0, seq_cap] set TQ_DEV_LEN_RANGE and are clamped for the attention).
+ *     Then the output is that of tq_decode_attention over positions
+ *     [0, seq_lens[b]).
  *   - k_new, v_new: device [batch, kv_heads, head_dim], kv_dtype TQ_F32 or
  *     TQ_F16, 16-byte aligned.  The norms and codes of the appended token
  *     may differ from tq_encode_kv's by one fp16 ulp where the fp32 norm is
@@ -248,10 +251,13 @@ int tq_decode_step(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_cod
  * library, which every GPU that loads the library holds until exit.
  *   - Limit: when tq_decode_workspace_size(desc, q_heads, sparse_thr) exceeds
  *     TQ_NOALLOC_SCRATCH_BYTES it returns TQ_ERR_SCRATCH_LIMIT and launches
- *     nothing.  Other argument errors are those of tq_decode_attention.
+ *     nothing.  Other argument errors are those of tq_decode_attention; all
+ *     of them are found before any CUDA call is made.
  *   - Set-up: the first call on each device looks up the array's device
  *     address (with that device current); make that first call before any
- *     stream capture.  Later calls do no set-up.
+ *     stream capture.  Later calls do no set-up.  The address is kept for the
+ *     life of the process, so this entry point must not be called on a device
+ *     after cudaDeviceReset() has destroyed the context it was looked up in.
  *   - Sharing: every call on a device uses the same array, which keeps the
  *     last call's contents; each call clears the counters that must start at
  *     zero (one cudaMemsetAsync on `stream`, no allocation).  Calls whose
@@ -265,6 +271,21 @@ int tq_decode_attention_noalloc(const tq_kv_desc* desc, const tq_codebook* k_cb,
                                 const uint8_t* v_codes, const uint16_t* v_norms,
                                 const int32_t* seq_lens, float scale, float sparse_thr, float* out,
                                 uint32_t* dev_status, void* stream);
+
+/*
+ * tq_read_device_status -- read the device status word that the kernels OR
+ * their range errors into (TQ_DEV_* bits above): rows written outside the
+ * cache and skipped, lengths clamped, norms saturated.  The kernels never
+ * trap on such data; this call is how a caller (or a test) learns of it.
+ * dev_status: device pointer, 4-byte aligned, the word passed to the other
+ *   calls.  bits_out: host pointer that receives the word.
+ * Synchronous: copies the word on `stream` and waits for the stream, so the
+ * bits of every call queued before it are included.  The word is not
+ * cleared (the caller owns it).  Returns TQ_OK when no bit is set,
+ * TQ_ERR_DEVICE_BOUNDS when any is, TQ_ERR_INVALID_ARG for a null or
+ * misaligned pointer and TQ_ERR_CUDA if the copy fails.
+ */
+int tq_read_device_status(const uint32_t* dev_status, uint32_t* bits_out, void* stream);
 
 /* Static description of a status code. */
 const char* tq_status_string(int status);

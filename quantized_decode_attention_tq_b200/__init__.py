@@ -7,12 +7,13 @@ from ._lib import (TQ_DEV_LEN_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_POS_RANGE, TQ_
                    Codebook, KVDesc, TQError, lib)
 from .api import (Cache, alloc_cache, alloc_workspace, cache_shapes, codebook_arrays,
                   decode_attention, decode_attention_multi, decode_attention_noalloc, decode_step,
-                  decode_workspace_size, encode_kv, kv_desc, make_codebook, sign_vector)
+                  decode_workspace_size, encode_kv, kv_desc, make_codebook, read_device_status,
+                  sign_vector)
 
 __all__ = [
     "Cache", "Codebook", "KVDesc", "TQError", "TQ_F16", "TQ_F32", "TQ_DEV_LEN_RANGE",
     "TQ_DEV_NORM_OVERFLOW", "TQ_DEV_POS_RANGE", "alloc_cache", "alloc_workspace", "cache_shapes",
     "codebook_arrays", "decode_attention", "decode_attention_multi", "decode_attention_noalloc",
     "decode_step", "decode_workspace_size", "encode_kv", "kv_desc", "lib", "make_codebook",
-    "sign_vector",
+    "read_device_status", "sign_vector",
 ]

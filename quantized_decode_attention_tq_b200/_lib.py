@@ -8,7 +8,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 # TQ_LIBRARY may point at another build of the same C ABI (e.g. a tuning variant).
 LIB_PATH = os.environ.get("TQ_LIBRARY") or os.path.join(_HERE, "libtq_b200.so")
 
-TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_SCRATCH_LIMIT = range(6)
+(TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_DEVICE_BOUNDS,
+ TQ_ERR_SCRATCH_LIMIT) = range(7)
 TQ_NOALLOC_SCRATCH_BYTES = 64 << 20
 TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE = 1, 2, 4
 TQ_F32, TQ_F16 = 0, 1
@@ -51,6 +52,7 @@ SIGNATURES = {
     "tq_decode_attention_noalloc": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p,
                                             c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_float, c_float, c_void_p, c_void_p, c_void_p]),
+    "tq_read_device_status": (c_int, [c_void_p, c_void_p, c_void_p]),
     "tq_status_string": (ctypes.c_char_p, [c_int]),
 }
 

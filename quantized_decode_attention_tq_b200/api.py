@@ -11,7 +11,8 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from ._lib import (TQ_F16, TQ_F32, Codebook, KVDesc, check, lib)
+from ._lib import (TQ_ERR_DEVICE_BOUNDS, TQ_F16, TQ_F32, TQ_OK, Codebook, KVDesc, TQError, check,
+                   lib)
 
 
 def make_codebook(bits: int) -> Codebook:
@@ -192,3 +193,15 @@ def decode_attention_noalloc(cache: Cache, k_cb: Codebook, v_cb: Codebook, q, se
         _ptr(status, "status"), _stream(stream))
     check("tq_decode_attention_noalloc", st)
     return out
+
+
+def read_device_status(status, stream=None) -> int:
+    """The bits of a device status word (tq_read_device_status; synchronous).
+
+    Returns the TQ_DEV_* bits that the kernels OR-ed into ``status`` (a
+    one-element int32/uint32 CUDA tensor); 0 means no range error."""
+    bits = ctypes.c_uint32(0)
+    st = lib().tq_read_device_status(_ptr(status, "status"), ctypes.byref(bits), _stream(stream))
+    if st not in (TQ_OK, TQ_ERR_DEVICE_BOUNDS):
+        raise TQError("tq_read_device_status", st)
+    return int(bits.value)

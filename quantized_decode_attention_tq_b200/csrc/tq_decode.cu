@@ -957,8 +957,11 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     // ---- decode step: the CTA that holds a unit's last tile first writes the
     // sequence's new token (position len - 1) into the cache, K and V, one
     // warp per 128-block, so that its own copies read it.  Other head groups
-    // of the same kv-head write the same bytes.
-    if (MODE != kSparseV && p.kv_new[0] != nullptr && seg_hi == nt && len > 0) {
+    // of the same kv-head write the same bytes.  A length outside
+    // [1, seq_cap] appends nothing: clamping it would overwrite a cached
+    // token (the range error is reported by the length scan).
+    if (MODE != kSparseV && p.kv_new[0] != nullptr && seg_hi == nt && len > 0 &&
+        __ldg(p.seq_lens + b) == len) {
       if (cw < 2 * NB) {
         append_block(p, cw / NB, cw % NB, (size_t)b * p.kv_heads + sg.kvh, cache_row + (len - 1), lane,
                      reinterpret_cast<uint32_t*>(res) + 16 * cw);

@@ -135,13 +135,15 @@ struct StepRows {
   uint16_t* v_norms;
 };
 
-int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
-                  int q_heads, int n_q, const void* q, int q_dtype,
-                  const uint8_t* k_codes, const uint16_t* k_norms,
-                  const uint8_t* v_codes, const uint16_t* v_norms,
-                  const int32_t* seq_lens, float scale, float sparse_thr, float* out,
-                  void* workspace, size_t workspace_bytes, uint32_t* dev_status,
-                  void* stream, const StepRows* step) {
+}  // namespace
+
+namespace tq {
+
+int validate_decode(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                    int q_heads, int n_q, const void* q, int q_dtype, const uint8_t* k_codes,
+                    const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
+                    const int32_t* seq_lens, float scale, float sparse_thr, const float* out,
+                    const uint32_t* dev_status) {
   int st = check_desc(desc);
   if (st != TQ_OK) return st;
   if (desc->batch > tq::kMaxBatch || desc->head_dim > tq::kMaxDecodeHeadDim) return TQ_ERR_UNSUPPORTED;
@@ -160,6 +162,23 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
   if (!std::isfinite(scale) || std::isnan(sparse_thr)) return TQ_ERR_INVALID_ARG;
   if ((st = check_codebook(k_cb, desc->k_bits)) != TQ_OK) return st;
   if ((st = check_codebook(v_cb, desc->v_bits)) != TQ_OK) return st;
+  return TQ_OK;
+}
+
+}  // namespace tq
+
+namespace {
+
+int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                  int q_heads, int n_q, const void* q, int q_dtype,
+                  const uint8_t* k_codes, const uint16_t* k_norms,
+                  const uint8_t* v_codes, const uint16_t* v_norms,
+                  const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                  void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                  void* stream, const StepRows* step) {
+  int st = tq::validate_decode(desc, k_cb, v_cb, q_heads, n_q, q, q_dtype, k_codes, k_norms, v_codes,
+                               v_norms, seq_lens, scale, sparse_thr, out, dev_status);
+  if (st != TQ_OK) return st;
   if (step) {
     if (step->kv_dtype != TQ_F32 && step->kv_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
     if (!step->k_new || !step->v_new || !aligned(step->k_new, 16) || !aligned(step->v_new, 16))
@@ -346,6 +365,17 @@ int tq_decode_step(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_cod
                        &step);
 }
 
+int tq_read_device_status(const uint32_t* dev_status, uint32_t* bits_out, void* stream) {
+  if (!dev_status || !bits_out || !aligned(dev_status, 4)) return TQ_ERR_INVALID_ARG;
+  uint32_t bits = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&bits, dev_status, sizeof(bits), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TQ_ERR_CUDA;
+  *bits_out = bits;
+  return bits ? TQ_ERR_DEVICE_BOUNDS : TQ_OK;
+}
+
 const char* tq_status_string(int status) {
   switch (status) {
     case TQ_OK: return "ok";
@@ -353,6 +383,7 @@ const char* tq_status_string(int status) {
     case TQ_ERR_UNSUPPORTED: return "unsupported configuration";
     case TQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case TQ_ERR_CUDA: return "CUDA runtime error";
+    case TQ_ERR_DEVICE_BOUNDS: return "the device status word reports a range error (clamped or skipped rows)";
     case TQ_ERR_SCRATCH_LIMIT: return "request needs more than the built-in no-alloc scratch array";
     default: return "unknown status";
   }

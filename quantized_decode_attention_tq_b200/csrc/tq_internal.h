@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/tq.h"
+
 namespace tq {
 
 constexpr int kBlock = 128;        // elements per rotated/quantised block
@@ -73,5 +75,13 @@ DecodeWorkspace decode_workspace_layout(int batch, int kv_heads, int q_heads, in
                                         int seq_cap, bool sparse);
 
 int launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+// Host-side argument checks shared by every decode entry point (no CUDA call;
+// the workspace is checked separately by the entry points that take one).
+int validate_decode(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                    int q_heads, int n_q, const void* q, int q_dtype, const uint8_t* k_codes,
+                    const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
+                    const int32_t* seq_lens, float scale, float sparse_thr, const float* out,
+                    const uint32_t* dev_status);
 
 }  // namespace tq

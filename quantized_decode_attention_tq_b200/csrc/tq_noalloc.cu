@@ -51,11 +51,15 @@ extern "C" int tq_decode_attention_noalloc(const tq_kv_desc* desc, const tq_code
                                            const uint16_t* v_norms, const int32_t* seq_lens,
                                            float scale, float sparse_thr, float* out,
                                            uint32_t* dev_status, void* stream) {
+  // Every argument check runs before the first CUDA call.
+  int st = tq::validate_decode(desc, k_cb, v_cb, q_heads, 1, q, q_dtype, k_codes, k_norms, v_codes,
+                               v_norms, seq_lens, scale, sparse_thr, out, dev_status);
+  if (st != TQ_OK) return st;
   const size_t need = tq_decode_workspace_size(desc, q_heads, sparse_thr);
   if (need == 0) return TQ_ERR_INVALID_ARG;
   if (need > (size_t)TQ_NOALLOC_SCRATCH_BYTES) return TQ_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
-  int st = scratch_address(&scratch);
+  st = scratch_address(&scratch);
   if (st != TQ_OK) return st;
   // The merge counters at the start of the workspace must be zero; the array
   // keeps whatever the previous call left, so clear them on the caller's stream.

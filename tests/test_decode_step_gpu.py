@@ -132,3 +132,37 @@ def test_decode_step_agrees_with_append_then_decode():
     tq.decode_attention(c2, kcb, vcb, to_dev(w.q), to_dev(np.asarray(lens, dtype=np.int32)), w.scale, out, ws)
     torch.cuda.synchronize()
     assert rel_err(o_step, out.cpu().numpy().astype(np.float64)) <= 1e-3
+
+
+def test_decode_step_length_beyond_cache_appends_nothing():
+    """seq_lens[b] = seq_cap + 1 is a range error: the status bit is set, the
+    attention runs over the clamped length, and no cached token -- in
+    particular the last one, where a clamped append would land -- changes."""
+    torch = torch_mod()
+    w = inputs.make("gqa", batch=2, seq=64)
+    desc = tq.kv_desc(2, w.kv_heads, 128, 64, w.k_bits, w.v_bits, w.sign_seed)
+    kcb, vcb = tq.make_codebook(w.k_bits), tq.make_codebook(w.v_bits)
+    cache = tq.alloc_cache(desc)
+    tq.encode_kv(cache, kcb, vcb, to_dev(w.k), to_dev(w.v))
+    before = host(cache)
+    lens = np.array([65, 40], dtype=np.int32)
+    rng = np.random.default_rng(9)
+    k_new = (rng.standard_normal((2, w.kv_heads, 128)) * 3).astype(np.float16)
+    v_new = (rng.standard_normal((2, w.kv_heads, 128)) * 3).astype(np.float16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((2, w.q_heads, 128), float("nan"), dtype=torch.float32, device="cuda")
+    ws = tq.alloc_workspace(desc, w.q_heads)
+    tq.decode_step(cache, kcb, vcb, to_dev(w.q), to_dev(k_new), to_dev(v_new), to_dev(lens), w.scale,
+                   out, ws, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == tq.TQ_DEV_LEN_RANGE
+    after = host(cache)
+    # sequence 0: nothing written; sequence 1: only position 39 changed
+    for a, b in zip(before, after):
+        assert np.array_equal(a[0], b[0])
+        keep = np.ones(a.shape[2], dtype=bool)
+        keep[39] = False
+        assert np.array_equal(a[1][:, keep], b[1][:, keep])
+    kc, kn, vc, vn = after
+    o_ref = oracle_decode(w.q, kc, kn, vc, vn, [64, 40], w.scale, w.k_bits, w.v_bits, 0.0)
+    check_decode(out.cpu().numpy().astype(np.float64), o_ref)

@@ -24,7 +24,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol():
     names = _header_functions()
-    assert len(names) == 9
+    assert len(names) == 10
     lib = tq.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -199,3 +199,44 @@ def test_cache_shapes_give_b_plus_one_eighth_bits():
         norm_bytes = 2 * int(np.prod(s["k_norms"]))
         values = 2 * 3 * 10 * 256
         assert (code_bytes + norm_bytes) * 8 / values == b + 16 / 128
+
+
+def test_noalloc_checks_arguments_before_any_cuda_call():
+    """Every argument error of the no-alloc entry point is found on the host,
+    before the scratch array is looked up: here, with no GPU at all, a bad
+    call returns its own status, never TQ_ERR_CUDA."""
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+
+    def call(desc=d, hq=8, q=GOOD, qd=1, lens=GOOD, out=GOOD, scale=0.1, thr=0.0, kcb=cb3, status=None):
+        return lib.tq_decode_attention_noalloc(ctypes.byref(desc), ctypes.byref(kcb), ctypes.byref(cb2), hq,
+                                               _fake(q) if q else None, qd, _fake(GOOD), _fake(GOOD),
+                                               _fake(GOOD), _fake(GOOD), _fake(lens) if lens else None,
+                                               scale, thr, _fake(out) if out else None,
+                                               _fake(status) if status else None, None)
+
+    assert call(q=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(qd=9) == _lib.TQ_ERR_INVALID_ARG
+    assert call(hq=7) == _lib.TQ_ERR_INVALID_ARG
+    assert call(lens=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(out=GOOD + 4) == _lib.TQ_ERR_INVALID_ARG
+    assert call(scale=math.nan) == _lib.TQ_ERR_INVALID_ARG
+    assert call(kcb=cb2) == _lib.TQ_ERR_INVALID_ARG
+    assert call(status=GOOD + 2) == _lib.TQ_ERR_INVALID_ARG
+    assert call(desc=tq.kv_desc(2, 2, 128, 63, 3, 2)) == _lib.TQ_ERR_UNSUPPORTED
+    big = tq.kv_desc(64, 8, 256, 65536, 3, 3)
+    assert lib.tq_decode_attention_noalloc(ctypes.byref(big), ctypes.byref(cb3), ctypes.byref(cb3), 32,
+                                           _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                           _fake(GOOD), _fake(GOOD), 0.1, 1e-5, _fake(GOOD), None,
+                                           None) == _lib.TQ_ERR_SCRATCH_LIMIT
+
+
+def test_read_device_status_argument_errors():
+    lib = tq.lib()
+    bits = ctypes.c_uint32(0)
+    assert lib.tq_read_device_status(None, ctypes.byref(bits), None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_read_device_status(_fake(GOOD), None, None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_read_device_status(_fake(GOOD + 2), ctypes.byref(bits), None) == _lib.TQ_ERR_INVALID_ARG
+    assert lib.tq_status_string(_lib.TQ_ERR_DEVICE_BOUNDS).decode().startswith("the device status")
+    assert lib.tq_status_string(_lib.TQ_ERR_SCRATCH_LIMIT).decode().startswith("request needs")
