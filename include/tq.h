@@ -68,6 +68,9 @@ typedef enum {
 #define TQ_DEV_POS_RANGE 1u      /* encode row outside [0, seq_cap): skipped */
 #define TQ_DEV_NORM_OVERFLOW 2u  /* block norm above fp16 max: saturated     */
 #define TQ_DEV_LEN_RANGE 4u      /* seq_lens[b] outside [0, seq_cap]: clamped */
+#define TQ_DEV_INTERNAL 8u       /* internal failure: the decode kernel's
+                                    shared-memory plan did not match the device
+                                    (nothing was computed; outputs are invalid) */
 
 typedef enum { TQ_F32 = 0, TQ_F16 = 1 } tq_dtype;
 
@@ -159,6 +162,8 @@ size_t tq_decode_workspace_size(const tq_kv_desc* desc, int q_heads, float spars
  * above 8 run in slices of 8).
  * q: device [batch, q_heads, head_dim], q_dtype TQ_F32 or TQ_F16.
  *    q_heads must be a multiple of kv_heads.
+ * scale: the softmax scale, finite and > 0 (1/sqrt(head_dim) in the usual
+ *    attention); other values give TQ_ERR_INVALID_ARG.
  * seq_lens: device int32 [batch]; values are clamped to [0, seq_cap]
  *    (TQ_DEV_LEN_RANGE).  A length of 0 gives an all-zero output row.
  * out: device fp32 [batch, q_heads, head_dim].

@@ -11,7 +11,7 @@ LIB_PATH = os.environ.get("TQ_LIBRARY") or os.path.join(_HERE, "libtq_b200.so")
 (TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_DEVICE_BOUNDS,
  TQ_ERR_SCRATCH_LIMIT) = range(7)
 TQ_NOALLOC_SCRATCH_BYTES = 64 << 20
-TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE = 1, 2, 4
+TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE, TQ_DEV_INTERNAL = 1, 2, 4, 8
 TQ_F32, TQ_F16 = 0, 1
 TQ_MAX_QUERY_TOKENS = 16
 

@@ -1,0 +1,11 @@
+// Decode-attention kernels for 3-bit K codes (every V bit width, head_dim
+// 128 and 256, every mode and group width); the kernel is in
+// tq_decode_kernel.cuh.
+
+#include "tq_decode_kernel.cuh"
+
+namespace tq {
+
+int launch_decode_k3(DecodeParams& p, cudaStream_t stream) { return dec::dispatch_kb<3>(p, stream); }
+
+}  // namespace tq

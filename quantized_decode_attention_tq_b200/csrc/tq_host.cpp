@@ -108,8 +108,8 @@ DecodeWorkspace decode_workspace_layout(int batch, int kv_heads, int q_heads, in
   const size_t units = (size_t)batch * kv_heads * n_hg;
   const size_t slots = kMaxCtas + units;
   size_t off = 0;
-  w.tickets_off = off;
-  off = align_up(off + units * sizeof(uint32_t), 256);
+  w.tickets_off = off;  // one count per (unit, head of the unit's group)
+  off = align_up(off + units * kMaxGroup * sizeof(uint32_t), 256);
   w.ml_off = off;
   off = align_up(off + slots * kMaxGroup * 2 * sizeof(float), 256);
   w.acc_off = off;
@@ -159,7 +159,7 @@ int validate_decode(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_co
       !aligned(v_norms, 4) || !aligned(seq_lens, 4) || !aligned(out, 16))
     return TQ_ERR_INVALID_ARG;
   if (dev_status && !aligned(dev_status, 4)) return TQ_ERR_INVALID_ARG;
-  if (!std::isfinite(scale) || std::isnan(sparse_thr)) return TQ_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.0f) || std::isnan(sparse_thr)) return TQ_ERR_INVALID_ARG;
   if ((st = check_codebook(k_cb, desc->k_bits)) != TQ_OK) return st;
   if ((st = check_codebook(v_cb, desc->v_bits)) != TQ_OK) return st;
   return TQ_OK;

@@ -34,6 +34,22 @@ struct EncodeParams {
 
 int launch_encode(const EncodeParams& p, cudaStream_t stream);
 
+constexpr int kDecodeWarps = 16;   // warps of one persistent decode CTA (one CTA per SM)
+
+// Shared-memory plan of a decode launch, computed on the host.  Every
+// address is an absolute shared-window address; the kernel checks that its
+// dynamic shared memory starts at `base` before using any of them.
+struct SmemPlan {
+  uint32_t base;                  // shared-window address of dynamic shared memory
+  uint32_t bytes;                 // dynamic shared memory requested
+  uint32_t lut_k, lut_v;          // code tables (byte tables: 64 KiB region + 0 / + 128)
+  uint32_t ring[kDecodeWarps];    // each warp's ring of tile slots (also its partial)
+  uint32_t res, misc, prefix;
+  uint32_t depth, slot_bytes;     // slots per ring, bytes per slot
+  uint32_t kc_off[4], vc_off[4];  // K / V codes of tokens 4j..4j+3 within a slot
+  uint32_t kn_off, vn_off;        // K / V norms within a slot
+};
+
 // Decode launch parameters.
 struct DecodeParams {
   const void* q;
@@ -46,7 +62,7 @@ struct DecodeParams {
   float* out;
   uint32_t* status;
   // workspace views
-  uint32_t* tickets;   // [units]
+  uint32_t* tickets;   // [units][kMaxGroup] tiles counted per (unit, head)
   float* slot_ml;      // [(kMaxCtas + units) * kMaxGroup * 2]
   float* slot_acc;     // [(kMaxCtas + units) * kMaxGroup * head_dim]
   float* scores;       // sparse only: [B, Hq, seq_cap] (log2-domain scores)
@@ -65,6 +81,7 @@ struct DecodeParams {
   uint8_t* app_codes[2];
   uint16_t* app_norms[2];
   float pos_bounds[2][7];  // positive decision boundaries of K and V, ascending
+  SmemPlan sm;        // filled by the launcher
 };
 
 // Workspace layout shared by the size query and the launcher.

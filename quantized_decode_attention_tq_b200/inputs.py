@@ -60,13 +60,18 @@ class Workload:
 
 
 def make(name: str, seed: int = 0, batch: int | None = None, seq: int | None = None,
-         ragged: tuple | None = None, with_q: bool = True) -> Workload:
+         ragged: tuple | None = None, with_q: bool = True, dist: str | None = None) -> Workload:
     """Generate workload ``name`` (optionally with a reduced batch / length).
 
     ``seq`` overrides the cache length (and the ragged range is scaled to it
-    unless ``ragged`` is given explicitly).
+    unless ``ragged`` is given explicitly).  ``dist`` overrides the K/V
+    distribution: "normal" or "outlier_t4" (the encode-only workload's
+    outlier-channel K and Student-t(4) V) at the workload's own shapes.
     """
     cfg = dict(WORKLOADS[name])
+    if dist is not None:
+        assert dist in ("normal", "outlier_t4"), dist
+        cfg["dist"] = dist
     bsz = batch if batch is not None else cfg["batch"]
     seq_cap = seq if seq is not None else cfg["seq"]
     rng = np.random.default_rng(seed)

@@ -138,7 +138,7 @@ def test_decode_repeatable_and_workspace_reuse():
     o2, _ = gpu_decode(cache, kcb, vcb, w.q, w.seq_lens, w.scale, workspace=ws, reps=3)
     assert np.array_equal(o1, o2)
     units = w.batch * w.kv_heads
-    assert torch.all(ws[: 4 * units] == 0).item()
+    assert torch.all(ws[: 4 * units * 8] == 0).item()  # one count per (unit, head slot)
 
 
 # ---------------------------------------------------------------- full size --
@@ -179,3 +179,38 @@ def test_decode_full_long_sampled(sparse):
 def test_decode_full_ragged_sampled():
     w = inputs.make("ragged")
     _full_sampled(w, [(0, 1), (3, 3)], w.sparse_thr)
+
+
+# ------------------------------------------------- heavy tails and peaks --
+
+@pytest.mark.parametrize("name,seq", [("gqa", 600), ("ragged", 700)])
+def test_decode_heavy_tailed_kv(name, seq):
+    """The encode-only workload's distributions through decode: K with
+    LogNormal per-channel scales and 2 % of channels x20 (block norms up to
+    ~100x the Gaussian ones), V ~ Student-t(4), at D128 and D256."""
+    w = inputs.make(name, batch=2, seq=seq, dist="outlier_t4")
+    w.seq_lens = np.array([seq, seq // 2 + 3], dtype=np.int32)
+    _run(w)
+    _run(w, sparse_thr=2e-3)
+
+
+@pytest.mark.parametrize("pos", ["first", "middle", "last"])
+@pytest.mark.parametrize("gain", [30.0, 60.0])
+def test_decode_peaked_attention(pos, gain):
+    """One cached key dominates: q_h = gain * k_j / |k_j| (scores of position j
+    about gain, the rest ~N(0, gain^2 / D)).  The running maximum jumps by far
+    more than the lazy-rescale threshold inside a tile, and every CTA that
+    does not hold position j sees weights that vanish after the merge.  The
+    sequences span several CTAs each."""
+    w = inputs.make("gqa", batch=2, seq=6000)
+    w.seq_lens = np.array([6000, 4321], dtype=np.int32)
+    q = np.empty((2, w.q_heads, 128), dtype=np.float64)
+    g = w.q_heads // w.kv_heads
+    for b in range(2):
+        n = int(w.seq_lens[b])
+        j = {"first": 3, "middle": n // 2 + 5, "last": n - 1}[pos]
+        for h in range(w.q_heads):
+            k = w.k[b, h // g, j].astype(np.float64)
+            q[b, h] = gain * k / np.linalg.norm(k) * (1.0 if h % 2 == 0 else 0.5)
+    w.q = q.astype(np.float16)
+    _run(w)

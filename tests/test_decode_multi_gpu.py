@@ -88,3 +88,9 @@ def test_decode_multi_short_sequences():
     # sequences shorter than n_q: the first tokens see nothing and give zeros
     w = inputs.make("gqa", batch=3, seq=64)
     _check(w, 5, [3, 64, 0], seed=7)
+
+
+def test_decode_multi_sixteen_tokens():
+    # the largest n_q the ABI accepts: 64 (token, head) columns per kv-head
+    w = inputs.make("gqa", batch=2, seq=256)
+    _check(w, tq._lib.TQ_MAX_QUERY_TOKENS, [256, 90], seed=16)
