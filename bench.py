@@ -11,11 +11,16 @@ so every step does identical work.
 
 Default workload: GQA decode, B8, Hq32/Hkv8, D128, S32768, K3/V3, fp16 Q.
 The packed cache (210 MB) rotates over enough copies to exceed 3x L2, so no
-timed step reads warm L2.  Also reported: the encoder alone on the encode-only
-workload (B8, Hkv8, D128, S32768 fp16 in, K3/V2).
+timed step reads warm L2.  Beside the timed steps the line reports the same
+steps replayed for at least a second (``sustained``), the other decode
+configurations with the same step (``workloads``: toy, long-context with
+sparse-V off and on, ragged wide-head), multi-token queries, and the encoder
+alone on the encode-only workload (B8, Hkv8, D128, S32768 fp16 in, K3/V2);
+``--encode-only`` runs only the last (for profiling).
 
-Multi-GPU: one process per GPU (torchrun); each rank serves its own batch
-(weak scaling, no collective on the data path); time = max over ranks.
+Multi-GPU: one process per GPU (torchrun, or spawned here when ``--gpus N``
+is given without a launcher); each rank serves its own batch (weak scaling,
+no collective on the data path); time = max over ranks.
 ``--impl reference`` times the CPU oracle on the same workload instead.
 """
 from __future__ import annotations
@@ -57,6 +62,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-encode", action="store_true", help="skip the encode-only measurement")
     ap.add_argument("--no-multi", action="store_true", help="skip the multi-token measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other decode configurations")
+    ap.add_argument("--sustain-s", type=float, default=1.0,
+                    help="seconds of extra replays reported beside the timed steps (0: off)")
+    ap.add_argument("--encode-only", action="store_true", help="only the encoder on the encode-only workload")
     return ap.parse_args(argv)
 
 
@@ -75,6 +84,7 @@ def workload(name, rank=0):
     w = inputs.make(base, seed=rank)
     if name == "long":
         w.sparse_thr = 0.0
+    w.name_key = name
     return w
 
 
@@ -173,12 +183,22 @@ def cpu_oracle_sample(w, kc, kn, vc, vn, units, budget_s=20.0):
 
 # ------------------------------------------------------------- traffic --
 
-def recorded_traffic(kernel_file, name):
+KERNEL_SOURCES = ("tq_decode_kernel.cuh", "tq_decode.cu")
+
+
+def kernel_sha():
+    """sha256 over the decode kernel's sources (what a profile was taken on)."""
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "quantized_decode_attention_tq_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic(name):
     """dram bytes per launch from a committed ncu summary, only if the kernel
-    source is unchanged since the capture (sha256 recorded beside it)."""
+    sources are unchanged since the capture (sha256 recorded beside it)."""
     path = os.path.join(ROOT, "profiles", name)
-    src = os.path.join(ROOT, "quantized_decode_attention_tq_b200", "csrc", kernel_file)
-    if not (os.path.exists(path) and os.path.exists(src)):
+    if not os.path.exists(path):
         return None
     fields = {}
     with open(path) as f:
@@ -186,8 +206,7 @@ def recorded_traffic(kernel_file, name):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if fields.get("kernel_sha256") != sha or "dram_bytes_per_launch" not in fields:
+    if fields.get("kernel_sha256") != kernel_sha() or "dram_bytes_per_launch" not in fields:
         return None
     return float(fields["dram_bytes_per_launch"])
 
@@ -237,11 +256,149 @@ def run_reference(args):
     return 0
 
 
+class StepBench:
+    """One workload on one GPU: its packed cache (built by the library's
+    encoder) in enough copies that every step reads cold memory, the step's
+    device inputs, and one CUDA graph per copy holding the step's launch(es).
+
+    A step is one decode step of every sequence: the newest K/V row is encoded
+    into the cache at seq_len - 1 inside the decode launch, then attention runs
+    over the whole cache (two launches with sparse-V)."""
+
+    def __init__(self, name, dev, seed=0):
+        import torch
+
+        import quantized_decode_attention_tq_b200 as tq
+        self.tq, self.torch, self.dev = tq, torch, dev
+        w = self.w = workload(name, seed)
+        self.desc = tq.kv_desc(w.batch, w.kv_heads, w.head_dim, w.seq_cap, w.k_bits, w.v_bits, w.sign_seed)
+        self.kcb, self.vcb = tq.make_codebook(w.k_bits), tq.make_codebook(w.v_bits)
+        cache0 = tq.alloc_cache(self.desc, dev)
+        tq.encode_kv(cache0, self.kcb, self.vcb, torch.from_numpy(w.k).to(dev), torch.from_numpy(w.v).to(dev))
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()  # the fp16 K/V staging copies are not needed on the device
+        self.cache0 = cache0
+        self.kvb = kv_bytes(w)
+        self.cache_bytes = sum(t.numel() * t.element_size() for t in
+                               (cache0.k_codes, cache0.k_norms, cache0.v_codes, cache0.v_norms))
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.n_copies = max(2, math.ceil(3 * l2 / max(self.cache_bytes, 1)) + 1)
+        self.caches = [cache0] + [tq.Cache(self.desc, cache0.k_codes.clone(), cache0.k_norms.clone(),
+                                           cache0.v_codes.clone(), cache0.v_norms.clone())
+                                  for _ in range(self.n_copies - 1)]
+        # step inputs: the newest row of every (batch, kv-head) and the query
+        self.lens_np = w.seq_lens.astype(np.int32)
+        pos_np = np.maximum(self.lens_np - 1, 0)
+        self.k_new_np = np.ascontiguousarray(w.k[np.arange(w.batch), :, pos_np])  # [B, Hkv, D]
+        self.v_new_np = np.ascontiguousarray(w.v[np.arange(w.batch), :, pos_np])
+        self.q = torch.from_numpy(w.q).to(dev)
+        self.k_new = torch.from_numpy(self.k_new_np).to(dev)
+        self.v_new = torch.from_numpy(self.v_new_np).to(dev)
+        self.lens = torch.from_numpy(self.lens_np).to(dev)
+        self.out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float32, device=dev)
+        self.ws = tq.alloc_workspace(self.desc, w.q_heads, w.sparse_thr, dev)
+        self.launches = 2 if w.sparse_thr > 0 else 1
+        for c in range(self.n_copies):  # eager warm-up (also primes the launch caches)
+            self.step(c)
+        torch.cuda.synchronize()
+        self.graphs = []
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for c in range(self.n_copies):
+                gs = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gs, stream=s):
+                    self.step(c)
+                self.graphs.append(gs)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+
+    def step(self, c):
+        w = self.w
+        self.tq.decode_step(self.caches[c], self.kcb, self.vcb, self.q, self.k_new, self.v_new, self.lens,
+                            w.scale, self.out, self.ws, sparse_thr=w.sparse_thr)
+
+    def replay(self, i):
+        self.graphs[i % self.n_copies].replay()
+
+    def time_steps(self, n, warmup=3):
+        """Mean device time of one step over n graph replays (CUDA events)."""
+        torch = self.torch
+        for i in range(warmup):
+            self.replay(i)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            self.replay(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    def summary(self, ms, peak):
+        gbs = self.kvb / (ms / 1e3) / 1e9
+        return {"workload": WORKLOAD_NAMES[self.w.name_key], "us_per_step": ms * 1e3,
+                "launches_per_step": self.launches, "kv_bytes": self.kvb, "hbm_gbs": gbs,
+                "frac_of_measured_hbm": gbs / peak, "kv_tokens_per_s": float(np.sum(self.w.seq_lens)) / (ms / 1e3)}
+
+    def release(self):
+        self.graphs = []
+        self.caches = []
+        self.cache0 = None
+        self.torch.cuda.synchronize()
+        self.torch.cuda.empty_cache()
+
+
+def encode_measure(dev, n_enc=20):
+    """The encoder alone on the encode-only workload (B8, Hkv8, D128, S32768,
+    fp16 in; K3 outlier-scaled Gaussian, V2 Student-t4): mean launch time."""
+    import torch
+
+    import quantized_decode_attention_tq_b200 as tq
+    from quantized_decode_attention_tq_b200 import inputs
+    we = inputs.make("encode", with_q=False)
+    de = tq.kv_desc(we.batch, we.kv_heads, we.head_dim, we.seq_cap, we.k_bits, we.v_bits)
+    ce = tq.alloc_cache(de, dev)
+    ke, ve = torch.from_numpy(we.k).to(dev), torch.from_numpy(we.v).to(dev)
+    kcb_e, vcb_e = tq.make_codebook(we.k_bits), tq.make_codebook(we.v_bits)
+    for _ in range(3):
+        tq.encode_kv(ce, kcb_e, vcb_e, ke, ve)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(n_enc):
+        tq.encode_kv(ce, kcb_e, vcb_e, ke, ve)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    enc_ms = x0.elapsed_time(x1) / n_enc
+    n_blocks = we.batch * we.kv_heads * we.seq_cap
+    enc_bytes = ke.numel() * 2 * 2 + n_blocks * ((16 * we.k_bits + 2) + (16 * we.v_bits + 2))
+    peak, _ = measured_peaks()
+    info = {"workload": "encode-only B8 Hkv8 D128 S32768 fp16 in, K3 (outlier-scaled "
+                        "Gaussian) / V2 (Student-t4)",
+            "gbs": enc_bytes / (enc_ms / 1e3) / 1e9, "us": enc_ms * 1e3,
+            "bytes": enc_bytes, "frac_of_measured_hbm": enc_bytes / (enc_ms / 1e3) / 1e9 / peak,
+            "l2": "1.25 GB streamed per launch (> L2)"}
+    del ce, ke, ve
+    torch.cuda.empty_cache()
+    return info
+
+
+def run_encode_only(args):
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    print(json.dumps({"encode": encode_measure(dev, n_enc=max(1, args.steps))}), flush=True)
+    return 0
+
+
 def run_tq(args):
     import torch
     import torch.distributed as dist
-
-    import quantized_decode_attention_tq_b200 as tq
 
     from quantized_decode_attention_tq_b200 import dist as tqd
     rank, local, world = tqd.rank_info()
@@ -263,65 +420,14 @@ def run_tq(args):
     def allsum(x):
         return tqd.reduce_sum(x, dev)
 
-    w = workload(args.workload, tqd.workload_seed(rank))
-    desc = tq.kv_desc(w.batch, w.kv_heads, w.head_dim, w.seq_cap, w.k_bits, w.v_bits, w.sign_seed)
-    kcb, vcb = tq.make_codebook(w.k_bits), tq.make_codebook(w.v_bits)
-
-    # ---- build the packed cache with the library's encoder, then copies ----
-    cache0 = tq.alloc_cache(desc, dev)
-    tq.encode_kv(cache0, kcb, vcb, torch.from_numpy(w.k).to(dev), torch.from_numpy(w.v).to(dev))
-    torch.cuda.synchronize()
-    torch.cuda.empty_cache()  # the fp16 K/V staging copies are not needed on the device
-    kvb = kv_bytes(w)
-    cache_bytes = sum(t.numel() * t.element_size() for t in
-                      (cache0.k_codes, cache0.k_norms, cache0.v_codes, cache0.v_norms))
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    n_copies = max(2, math.ceil(3 * l2 / max(cache_bytes, 1)) + 1)
-    caches = [cache0] + [tq.Cache(desc, cache0.k_codes.clone(), cache0.k_norms.clone(),
-                                  cache0.v_codes.clone(), cache0.v_norms.clone())
-                         for _ in range(n_copies - 1)]
-
-    # step inputs: the newest row of every (batch, kv-head) and the query
-    lens_np = w.seq_lens.astype(np.int32)
-    pos_np = (lens_np - 1).astype(np.int32)
-    k_new_np = np.ascontiguousarray(w.k[np.arange(w.batch), :, pos_np])  # [B, Hkv, D]
-    v_new_np = np.ascontiguousarray(w.v[np.arange(w.batch), :, pos_np])
-    q = torch.from_numpy(w.q).to(dev)
-    k_new = torch.from_numpy(k_new_np).to(dev)
-    v_new = torch.from_numpy(v_new_np).to(dev)
-    lens = torch.from_numpy(lens_np).to(dev)
-    out = torch.empty(w.batch, w.q_heads, w.head_dim, dtype=torch.float32, device=dev)
-    ws = tq.alloc_workspace(desc, w.q_heads, w.sparse_thr, dev)
-    decode_launches = 2 if w.sparse_thr > 0 else 1
-
-    def step(c):
-        # one decode step: the newest token of every sequence is encoded into
-        # the cache at lens - 1 inside the decode launch, then attended over
-        tq.decode_step(caches[c], kcb, vcb, q, k_new, v_new, lens, w.scale, out, ws,
-                       sparse_thr=w.sparse_thr)
-
-    for c in range(n_copies):  # eager warm-up (also primes the launch caches)
-        step(c)
-    torch.cuda.synchronize()
-
-    # ---- CUDA graphs: one per cache copy, holding the step's launch(es) ------
-    g_step = []
-    s = torch.cuda.Stream(device=dev)
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        for c in range(n_copies):
-            gs = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gs, stream=s):
-                step(c)
-            g_step.append(gs)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-
+    peak, peak_kind = measured_peaks()
+    sb = StepBench(args.workload, dev, tqd.workload_seed(rank))
+    w, n_copies = sb.w, sb.n_copies
     for i in range(args.warmup):
-        g_step[i % n_copies].replay()
+        sb.replay(i)
     torch.cuda.synchronize()
 
-    # ---- timed region -------------------------------------------------------
+    # ---- timed region: exactly `steps` steps, barrier + sync on both sides ----
     stream = torch.cuda.current_stream()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -334,7 +440,7 @@ def run_tq(args):
     ev0.record(stream)
     for i in range(args.steps):
         ea[i].record(stream)
-        g_step[i % n_copies].replay()
+        sb.replay(i)
         eb[i].record(stream)
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -347,19 +453,40 @@ def run_tq(args):
     tokens_step = allsum(float(np.sum(w.seq_lens)))
     value = tokens_step / (ms / 1e3)
 
+    # ---- the same steps replayed for at least a second (steadier per-step
+    # time and a full clock record), beside the contract's timed steps -------
+    sustained = None
+    if args.sustain_s > 0:
+        n_long = max(args.steps, int(math.ceil(args.sustain_s / max(ms / 1e3, 1e-6))))
+        barrier()
+        torch.cuda.synchronize()
+        sampler2 = ClockSampler(local)
+        time.sleep(0.3)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(n_long):
+            sb.replay(i)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        clocks2 = sampler2.stop()
+        barrier()
+        ms_long = allmax(s0.elapsed_time(s1) / n_long)
+        sustained = {"steps": n_long, "ms_per_step": ms_long, "seconds": ms_long * n_long / 1e3,
+                     "value": tokens_step / (ms_long / 1e3), "clocks": clocks2}
+
     # ---- end to end through the public API with host buffers ---------------
     h2d, d2h = step_io_bytes(w)
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
-    q_h, k_h, v_h, l_h = pin(w.q), pin(k_new_np), pin(v_new_np), pin(lens_np)
-    out_h = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    q_h, k_h, v_h, l_h = pin(w.q), pin(sb.k_new_np), pin(sb.v_new_np), pin(sb.lens_np)
+    out_h = torch.empty(sb.out.shape, dtype=torch.float32).pin_memory()
 
     def e2e_step(c):
-        q.copy_(q_h, non_blocking=True)
-        k_new.copy_(k_h, non_blocking=True)
-        v_new.copy_(v_h, non_blocking=True)
-        lens.copy_(l_h, non_blocking=True)
-        step(c)
-        out_h.copy_(out, non_blocking=True)
+        sb.q.copy_(q_h, non_blocking=True)
+        sb.k_new.copy_(k_h, non_blocking=True)
+        sb.v_new.copy_(v_h, non_blocking=True)
+        sb.lens.copy_(l_h, non_blocking=True)
+        sb.step(c)
+        out_h.copy_(sb.out, non_blocking=True)
 
     for i in range(max(3, args.warmup)):
         e2e_step(i % n_copies)
@@ -378,23 +505,24 @@ def run_tq(args):
     # ---- multi-token queries on the same caches (n_q causal query tokens) ---
     multi_info = None
     if rank == 0 and not args.no_multi:
+        tq = sb.tq
         try:
             multi_info = {"workload": "the same caches and lengths; n_q query tokens per sequence "
                                       "(its last n_q positions, causal)", "us_per_launch": {},
                           "us_per_query_token": {}}
             for n_q in (2, 4):
-                qm = torch.randn(w.batch, n_q, w.q_heads, w.head_dim, device=dev).to(q.dtype)
+                qm = torch.randn(w.batch, n_q, w.q_heads, w.head_dim, device=dev).to(sb.q.dtype)
                 om = torch.empty(w.batch, n_q, w.q_heads, w.head_dim, dtype=torch.float32, device=dev)
-                wsm = tq.alloc_workspace(desc, w.q_heads * n_q, w.sparse_thr, dev)
+                wsm = tq.alloc_workspace(sb.desc, w.q_heads * n_q, w.sparse_thr, dev)
                 for i in range(3):
-                    tq.decode_attention_multi(caches[i % n_copies], kcb, vcb, qm, lens, w.scale, om, wsm,
-                                              sparse_thr=w.sparse_thr)
+                    tq.decode_attention_multi(sb.caches[i % n_copies], sb.kcb, sb.vcb, qm, sb.lens, w.scale, om,
+                                              wsm, sparse_thr=w.sparse_thr)
                 m0 = torch.cuda.Event(enable_timing=True)
                 m1 = torch.cuda.Event(enable_timing=True)
                 m0.record(stream)
                 for i in range(10):
-                    tq.decode_attention_multi(caches[i % n_copies], kcb, vcb, qm, lens, w.scale, om, wsm,
-                                              sparse_thr=w.sparse_thr)
+                    tq.decode_attention_multi(sb.caches[i % n_copies], sb.kcb, sb.vcb, qm, sb.lens, w.scale, om,
+                                              wsm, sparse_thr=w.sparse_thr)
                 m1.record(stream)
                 torch.cuda.synchronize()
                 us = m0.elapsed_time(m1) / 10 * 1e3
@@ -404,63 +532,55 @@ def run_tq(args):
         except Exception as e:  # reported, never fatal to the benchmark line
             multi_info = {"error": f"{type(e).__name__}: {e}"}
 
-    # ---- encoder alone on the encode-only workload -------------------------
-    encode_info = None
-    if not args.no_encode and rank == 0:
-        from quantized_decode_attention_tq_b200 import inputs
-        del caches, g_step
-        torch.cuda.empty_cache()
-        we = inputs.make("encode", with_q=False)
-        de = tq.kv_desc(we.batch, we.kv_heads, we.head_dim, we.seq_cap, we.k_bits, we.v_bits)
-        ce = tq.alloc_cache(de, dev)
-        ke, ve = torch.from_numpy(we.k).to(dev), torch.from_numpy(we.v).to(dev)
-        kcb_e, vcb_e = tq.make_codebook(we.k_bits), tq.make_codebook(we.v_bits)
-        for _ in range(3):
-            tq.encode_kv(ce, kcb_e, vcb_e, ke, ve)
-        torch.cuda.synchronize()
-        n_enc = 20
-        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        x0.record(stream)
-        for _ in range(n_enc):
-            tq.encode_kv(ce, kcb_e, vcb_e, ke, ve)
-        x1.record(stream)
-        torch.cuda.synchronize()
-        enc_ms = x0.elapsed_time(x1) / n_enc
-        n_blocks = we.batch * we.kv_heads * we.seq_cap
-        enc_bytes = ke.numel() * 2 * 2 + n_blocks * ((16 * we.k_bits + 2) + (16 * we.v_bits + 2))
-        peak, _ = measured_peaks()
-        encode_info = {"workload": "encode-only B8 Hkv8 D128 S32768 fp16 in, K3 (outlier-scaled "
-                                   "Gaussian) / V2 (Student-t4)",
-                       "gbs": enc_bytes / (enc_ms / 1e3) / 1e9, "us": enc_ms * 1e3,
-                       "bytes": enc_bytes, "frac_of_measured_hbm": enc_bytes / (enc_ms / 1e3) / 1e9 / peak,
-                       "l2": "1.25 GB streamed per launch (> L2)"}
-
     # ---- CPU oracle baseline (rank 0, N = 1) --------------------------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        kc = cache0.k_codes.cpu().numpy()
-        kn = cache0.k_norms.cpu().numpy().view(np.float16)
-        vc = cache0.v_codes.cpu().numpy()
-        vn = cache0.v_norms.cpu().numpy().view(np.float16)
+        kc = sb.cache0.k_codes.cpu().numpy()
+        kn = sb.cache0.k_norms.cpu().numpy().view(np.float16)
+        vc = sb.cache0.v_codes.cpu().numpy()
+        vn = sb.cache0.v_norms.cpu().numpy().view(np.float16)
         units = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
         v_cpu, threads, sample = cpu_oracle_sample(w, kc, kn, vc, vn, units, budget_s=15.0)
         cpu = {"value": v_cpu, "unit": "KV tokens/s", "cores": threads, "kind": "oracle", "sample": sample}
 
+    main_cfg = {"workload": WORKLOAD_NAMES[args.workload], "batch_per_gpu": w.batch,
+                "seq_len": w.seq_cap, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
+                "head_dim": w.head_dim, "k_bits": w.k_bits, "v_bits": w.v_bits,
+                "sparse_thr": w.sparse_thr, "parallelism": f"independent batches x{world}",
+                "l2": f"rotating {n_copies} cache copies of {sb.cache_bytes / 1e6:.0f} MB (> 3x L2)"}
+    kvb, launches = sb.kvb, sb.launches
+    sb.release()
+    del sb
+
+    # ---- the other decode configurations, same step, rank 0 -----------------
+    others = None
+    if rank == 0 and not args.no_workloads:
+        others = {}
+        for name in [n for n in ("toy", "long", "long_sparse", "ragged", "gqa") if n != args.workload]:
+            try:
+                ob = StepBench(name, dev, 0)
+                ms_o = ob.time_steps(max(20, args.steps), warmup=max(3, args.warmup))
+                others[name] = ob.summary(ms_o, peak)
+                ob.release()
+                del ob
+            except Exception as e:  # reported, never fatal to the benchmark line
+                others[name] = {"error": f"{type(e).__name__}: {e}"}
+
+    # ---- encoder alone on the encode-only workload -------------------------
+    encode_info = None
+    if not args.no_encode and rank == 0:
+        encode_info = encode_measure(dev)
+
     if rank == 0:
-        peak, peak_kind = measured_peaks()
         achieved = kvb / (dec_ms / 1e3) / 1e9
-        traffic = recorded_traffic("tq_decode.cu", f"decode_{args.workload}_traffic.txt")
+        traffic = recorded_traffic(f"decode_{args.workload}_traffic.txt")
         line = {
             "metric": METRIC, "value": value, "unit": "KV tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16xf16->f32 (tensor-core products of fp16 codewords, fp32 softmax/accumulate)",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAMES[args.workload], "batch_per_gpu": w.batch,
-                       "seq_len": w.seq_cap, "q_heads": w.q_heads, "kv_heads": w.kv_heads,
-                       "head_dim": w.head_dim, "k_bits": w.k_bits, "v_bits": w.v_bits,
-                       "sparse_thr": w.sparse_thr, "parallelism": f"independent batches x{world}",
-                       "l2": f"rotating {n_copies} cache copies of {cache_bytes / 1e6:.0f} MB (> 3x L2)"},
+            "config": main_cfg,
             "decode_us": dec_ms * 1e3, "hbm_gbs": achieved,
             "hbm_frac_of_8tbs": achieved / 8000.0,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -469,8 +589,10 @@ def run_tq(args):
                          "algorithmic_bytes_per_launch": kvb},
             "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * decode_launches,
+            "gpu_launches": args.steps * launches,
             "clocks": clocks,
+            "sustained": sustained,
+            "workloads": others,
             "encode": encode_info,
             "multi_token": multi_info,
             "cpu_baseline": cpu,
@@ -481,10 +603,26 @@ def run_tq(args):
     return 0
 
 
+def _rank_main(argv):
+    """Entry of one spawned rank (see main)."""
+    return run_tq(parse_args(argv))
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.encode_only:
+        return run_encode_only(args)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # --gpus N without a launcher: one process per GPU, spawned here with
+        # the torchrun environment (rank 0 prints the line)
+        from quantized_decode_attention_tq_b200 import dist as tqd
+        return tqd.launch_local(args.gpus, _rank_main, list(sys.argv[1:] if argv is None else argv))
+    from quantized_decode_attention_tq_b200 import dist as tqd
+    _, _, world = tqd.rank_info()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} rank(s)")
     return run_tq(args)
 
 

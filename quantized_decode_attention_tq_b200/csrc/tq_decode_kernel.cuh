@@ -370,12 +370,23 @@ __device__ __noinline__ void append_block(const DecodeParams& p, int side, int b
 // adds no segment.  Results do not depend on the split (each part is computed
 // and merged in a fixed order); it only moves where the CTAs end.
 
-// floor(a / b) for 0 <= a, 0 < b, both below 2^52: the double quotient is
-// within one of the exact one, and one integer step corrects it (a 64-bit
-// integer division is a long instruction sequence on the GPU).
-__device__ __forceinline__ long long fdiv(long long a, long long b) {
-  long long q = (long long)((double)a / (double)b);
-  if (q * b > a) --q; else if ((q + 1) * b <= a) ++q;
+// floor(a / b) for 0 <= a, 0 < b, both below 2^52, from the reciprocal
+// inv_b ~= 1 / b: the double estimate is within one of the exact quotient and
+// integer steps correct it (a 64-bit integer division, or a double division,
+// is a long instruction sequence on the GPU).
+__device__ __forceinline__ long long qdiv(long long a, long long b, double inv_b) {
+  long long q = (long long)((double)a * inv_b);
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;
+  return q;
+}
+// floor(a / b) when the quotient is below 2^20: a single-precision estimate
+// from the hardware reciprocal, then exact integer steps.
+__device__ __forceinline__ long long qdiv_small(long long a, long long b) {
+  long long q = (long long)((float)a * __frcp_rn((float)b));
+  if (q < 0) q = 0;
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;
   return q;
 }
 
@@ -383,15 +394,19 @@ struct Split {
   const int* prefix;  // [B+1] tiles per batch entry, exclusive prefix (shared memory)
   int B, UB;
   long long P, T, Ctot;
+  double invP, invCtot, invUB;
   __device__ Split(const int* pre, int batch, int ub, long long parts)
       : prefix(pre), B(batch), UB(ub), P(parts) {
     T = (long long)pre[batch] * ub;
     Ctot = (long long)ub * ((long long)pre[batch] + kSwitchTiles * batch);
+    invP = 1.0 / (double)P;
+    invCtot = Ctot > 0 ? 1.0 / (double)Ctot : 0.0;
+    invUB = 1.0 / (double)ub;
   }
   // first tile of part c (c = P gives T)
   __device__ long long start(long long c) const {
     if (c >= P) return T;
-    const long long y = fdiv(c * Ctot, P);
+    const long long y = qdiv(c * Ctot, P, invP);
     int bl = 0, bh = B;  // largest b with cost(b) <= y
     while (bh - bl > 1) {
       const int mid = (bl + bh) >> 1;
@@ -399,7 +414,7 @@ struct Split {
     }
     const long long nt = prefix[bl + 1] - prefix[bl];
     const long long rem = y - (long long)UB * (prefix[bl] + kSwitchTiles * bl);
-    const long long r = fdiv(rem, nt + kSwitchTiles), t = rem - r * (nt + kSwitchTiles);
+    const long long r = qdiv_small(rem, nt + kSwitchTiles), t = rem - r * (nt + kSwitchTiles);
     return (long long)UB * prefix[bl] + r * nt + min(t, nt);
   }
   // The part whose range holds tile x (0 <= x < T): the last c whose cost
@@ -412,9 +427,9 @@ struct Split {
     }
     const long long nt = prefix[bl + 1] - prefix[bl];
     const long long off = x - (long long)UB * prefix[bl];
-    const long long r = fdiv(off, nt), t = off - r * nt;
+    const long long r = qdiv_small(off, nt), t = off - r * nt;
     const long long F = (long long)UB * (prefix[bl] + kSwitchTiles * bl) + r * (nt + kSwitchTiles) + t;
-    const long long c = fdiv((F + 1) * P - 1, Ctot);
+    const long long c = qdiv((F + 1) * P - 1, Ctot, invCtot);
     return c < P - 1 ? c : P - 1;
   }
 };
@@ -468,10 +483,10 @@ struct Segment {
 };
 
 __device__ __forceinline__ Segment locate(long long x, long long hi, const int* prefix, int batch,
-                                          int UB, int n_hg, int G, int seq_cap,
+                                          int UB, double invUB, int n_hg, int G, int seq_cap,
                                           const int32_t* seq_lens) {
   Segment s;
-  const long long y = x / UB;  // in units of "tiles per batch entry"
+  const long long y = qdiv(x, UB, invUB);  // in units of "tiles per batch entry"
   int bl = 0, bh = batch;      // largest b with prefix[b] <= y
   while (bh - bl > 1) {
     const int mid = (bl + bh) >> 1;
@@ -480,7 +495,7 @@ __device__ __forceinline__ Segment locate(long long x, long long hi, const int* 
   s.b = bl;
   s.nt = prefix[bl + 1] - prefix[bl];
   const long long TB = (long long)prefix[bl] * UB;
-  s.r = (int)((x - TB) / s.nt);
+  s.r = (int)qdiv_small(x - TB, s.nt);
   s.Su = TB + (long long)s.r * s.nt;
   s.seg_lo = (int)(x - s.Su);
   s.seg_hi = (int)(min(hi, s.Su + s.nt) - s.Su);
@@ -668,30 +683,36 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     return ((size_t)b * p.n_q + vl / G) * p.q_heads + kvh * G + vl % G;
   };
 
-  // ---- tables -------------------------------------------------------------
-  auto fill_table = [&](int bits, const float* cent, uint32_t base, uint32_t half) {
+  // ---- code tables, filled by the threads [t_first, t_first + t_count) ------
+  auto fill_table = [&](int bits, const float* cent, uint32_t base, uint32_t half, int t_first, int t_count) {
+    const int t = tid - t_first;
     if (bits == 3) {  // 64 pairs x 32 lanes
-      for (int e = tid; e < 64 * 32; e += kThreads) {
+      for (int e = t; e < 64 * 32; e += t_count) {
         const int f = e >> 5;
-        st_s32(base + 4u * e, pack_half2(cent[f & 7], cent[f >> 3]));
+        *reinterpret_cast<uint32_t*>(gptr(base + 4u * e)) = pack_half2(cent[f & 7], cent[f >> 3]);
       }
     } else if (bits == 4) {  // 256 pairs x 32 lanes
-      for (int e = tid; e < 256 * 32; e += kThreads) {
+      for (int e = t; e < 256 * 32; e += t_count) {
         const int f = e >> 5, l = e & 31;
-        st_s32(base + 256u * f + half + 4u * l, pack_half2(cent[f & 15], cent[f >> 4]));
+        *reinterpret_cast<uint32_t*>(gptr(base + 256u * f + half + 4u * l)) = pack_half2(cent[f & 15], cent[f >> 4]);
       }
     } else {  // 2 bits: 256 quads x 16 lanes
-      for (int e = tid; e < 256 * 16; e += kThreads) {
+      for (int e = t; e < 256 * 16; e += t_count) {
         const int f = e >> 4, l = e & 15;
-        st_s64(base + 256u * f + half + 8u * l, pack_half2(cent[f & 3], cent[(f >> 2) & 3]),
-               pack_half2(cent[(f >> 4) & 3], cent[f >> 6]));
+        *reinterpret_cast<uint2*>(gptr(base + 256u * f + half + 8u * l)) =
+            make_uint2(pack_half2(cent[f & 3], cent[(f >> 2) & 3]), pack_half2(cent[(f >> 4) & 3], cent[f >> 6]));
       }
     }
   };
-  if constexpr (HASK) fill_table(KB, p.kcent, KB == 3 ? sm.lut_k : sm.lut_k & ~255u, KB == 3 ? 0u : (sm.lut_k & 128u));
-  if constexpr (HASV) fill_table(VB, p.vcent, VB == 3 ? sm.lut_v : sm.lut_v & ~255u, VB == 3 ? 0u : (sm.lut_v & 128u));
+  auto fill_tables = [&](int t_first, int t_count) {
+    if (tid < t_first || tid >= t_first + t_count) return;
+    if constexpr (HASK)
+      fill_table(KB, p.kcent, KB == 3 ? sm.lut_k : sm.lut_k & ~255u, KB == 3 ? 0u : (sm.lut_k & 128u), t_first, t_count);
+    if constexpr (HASV)
+      fill_table(VB, p.vcent, VB == 3 ? sm.lut_v : sm.lut_v & ~255u, VB == 3 ? 0u : (sm.lut_v & 128u), t_first, t_count);
+  };
+  bool tables_ready = false;  // filled during the first segment's query preparation
 
-  // ---- ring barriers ---------------------------------------------------------
   // ---- lengths: clamp, tiles per batch entry, exclusive prefix ------------
   {
     const int B = p.batch;
@@ -728,19 +749,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   const Split sp(prefix, p.batch, UB, gridDim.x);  // this launch's split
   const long long T = sp.T;
 
-  // ---- zero rows of empty sequences (only the V-producing passes) ---------
-  if constexpr (MODE != kScores) {
-    const long long rows = (long long)p.batch * p.n_q * p.q_heads;
-    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
-      const int b = (int)(row / ((long long)p.n_q * p.q_heads));
-      if (prefix[b + 1] == prefix[b]) {
-        for (int d = tid; d < D; d += kThreads) p.out[row * D + d] = 0.0f;
-      }
-    }
-  }
-  if (T == 0) return;
-
-  const long long lo = sp.start(blockIdx.x), hi = sp.start(blockIdx.x + 1);
+  const long long lo = T > 0 ? sp.start(blockIdx.x) : 0, hi = T > 0 ? sp.start(blockIdx.x + 1) : 0;
   const int cw = warp;
   const uint32_t wring_s = sm.ring[cw];  // this warp's ring
   const uint32_t slot_bytes = sm.slot_bytes;
@@ -798,6 +807,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   auto prep_q = [&](int b, int h0, int Gu, uint32_t (&qf)[NB][8][2], float (&qmul)[2]) {
     constexpr int kQRows = kDup ? 4 : kMaxGroup;
     float* qs = res;  // [kQRows] rows of scaled qhat (QScratch layout)
+    // the first segment's idle warps fill the code tables meanwhile
+    if (!tables_ready) fill_tables(32 * kQRows, kThreads - 32 * kQRows);
     for (int j = cw; j < kQRows; j += kCWarps) {
       float v[NB][4];
 #pragma unroll
@@ -848,6 +859,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         qf[blk][j][1] = pack_half2(q4.z, q4.w);
       }
     }
+    tables_ready = true;
     qmul[0] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g) & 3 : 2 * g]);
     qmul[1] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g + 1) & 3 : 2 * g + 1]);
     consumer_sync();  // res and qexp are reused after this
@@ -872,7 +884,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   };
 
   for (long long x = lo; x < hi;) {
-    const Segment sg = locate(x, hi, prefix, p.batch, UB, n_hg, Gv, p.seq_cap, p.seq_lens);
+    const Segment sg = locate(x, hi, prefix, p.batch, UB, sp.invUB, n_hg, Gv, p.seq_cap, p.seq_lens);
     const int b = sg.b, nt = sg.nt, unit = sg.unit, h0 = sg.h0, Gu = sg.Gu, len = sg.len;
     const int seg_lo = sg.seg_lo, seg_hi = sg.seg_hi;
     const long long Su = sg.Su;
@@ -952,6 +964,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     float lse2[2] = {0.0f, 0.0f};
     if constexpr (HASK) prep_q(b, h0, Gu, qf, qmul);
     if constexpr (MODE == kSparseV) {
+      if (!tables_ready) fill_tables(0, kThreads);
+      tables_ready = true;
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote; warp hd takes head hd
       const Split sp1(prefix, p.batch, UB, p1_ctas);
@@ -1394,6 +1408,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     x = Su + seg_hi;
   }
 
+
+  // ---- zero rows of empty sequences (only the V-producing passes; off the
+  // critical path, after the tiles) ---------------------------------------------
+  if constexpr (MODE != kScores) {
+    const long long rows = (long long)p.batch * p.n_q * p.q_heads;
+    for (long long row = blockIdx.x; row < rows; row += gridDim.x) {
+      const int b = (int)(row / ((long long)p.n_q * p.q_heads));
+      if (prefix[b + 1] == prefix[b]) {
+        for (int d = tid; d < D; d += kThreads) p.out[row * D + d] = 0.0f;
+      }
+    }
+  }
 }
 
 // --------------------------------------------------------------- launching --

@@ -46,3 +46,53 @@ def aggregate_throughput(units_per_rank: float, ms_per_step_per_rank: float, dev
     total = reduce_sum(units_per_rank, device)
     ms = reduce_max(ms_per_step_per_rank, device)
     return total / (ms / 1e3), ms, total
+
+
+def _free_port() -> int:
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _spawned(rank: int, world: int, port: int, fn, args):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    rc = fn(*args)
+    raise SystemExit(int(rc or 0))
+
+
+def launch_local(world: int, fn, *args, timeout_s: float = 1800.0) -> int:
+    """Run ``fn(*args)`` in ``world`` processes on this node, with the
+    environment torchrun would set (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_ADDR
+    127.0.0.1, MASTER_PORT); processes are spawned, not forked, so no CUDA
+    state is inherited.  Returns 0 when every rank exits 0; otherwise the
+    ranks still running are terminated and the first non-zero exit code is
+    returned."""
+    import time
+
+    import torch.multiprocessing as mp
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_spawned, args=(r, world, port, fn, args)) for r in range(world)]
+    for p in procs:
+        p.start()
+    deadline = time.monotonic() + timeout_s
+    rc = 0
+    for p in procs:
+        p.join(max(0.0, deadline - time.monotonic()))
+        if p.exitcode is None:
+            rc = rc or 124  # timed out
+        elif p.exitcode != 0:
+            rc = rc or p.exitcode
+        if rc:
+            break
+    for p in procs:
+        if p.is_alive():
+            p.terminate()
+            p.join(10)
+    return rc

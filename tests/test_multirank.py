@@ -52,3 +52,39 @@ def test_two_rank_aggregation():
     assert ms0 == ms1 == 3.0              # the slowest rank sets the time
     assert tot0 == tot1 == t0 + t1
     assert rate0 == rate1 == pytest.approx((t0 + t1) / 3e-3)
+
+
+def _launched_worker(path, value):
+    """A rank started by dist.launch_local: joins a gloo group from the
+    environment the launcher set and reduces through the benchmark helpers."""
+    import torch.distributed as dist
+    from datetime import timedelta
+    from quantized_decode_attention_tq_b200 import dist as tqd
+    dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    try:
+        r, lr, ws = tqd.rank_info()
+        total = tqd.reduce_sum(value + r)
+        mx = tqd.reduce_max(float(r))
+        with open(f"{path}.{r}", "w") as f:
+            f.write(f"{r} {lr} {ws} {total} {mx}")
+    finally:
+        dist.destroy_process_group()
+    return 0
+
+
+def _failing_worker(rank_to_fail):
+    import os
+    return 3 if int(os.environ["RANK"]) == rank_to_fail else 0
+
+
+def test_launch_local_runs_every_rank_with_the_torchrun_environment(tmp_path):
+    from quantized_decode_attention_tq_b200 import dist as tqd
+    path = str(tmp_path / "out")
+    assert tqd.launch_local(2, _launched_worker, path, 10.0, timeout_s=300) == 0
+    got = sorted(open(f"{path}.{r}").read().split() for r in range(2))
+    assert got == [["0", "0", "2", "21.0", "1.0"], ["1", "1", "2", "21.0", "1.0"]]
+
+
+def test_launch_local_reports_a_failing_rank():
+    from quantized_decode_attention_tq_b200 import dist as tqd
+    assert tqd.launch_local(2, _failing_worker, 1, timeout_s=300) == 3
