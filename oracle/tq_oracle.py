@@ -36,7 +36,10 @@ Readings taken where the pages are silent:
     boundary goes to the lower index; a zero block gives index L/2 - 1;
   * codes packed LSB-first into a little-endian bitstream of 16*b bytes;
   * sparse-V weight = normalised softmax weight exp(s - LSE); positions below
-    the threshold contribute zero and the rest are not renormalised.
+    the threshold contribute zero and the rest are not renormalised;
+  * V v3 (outlier-channel separation): a fixed set of k channels per kv-head
+    (largest mean square on calibration vectors) kept exactly as fp16, the
+    rest of the vector encoded as v1 (see encode_v3).
 """
 from __future__ import annotations
 
@@ -399,6 +402,85 @@ def attention_multi(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_lens, scale
                 if sparse_thr > 0:
                     w = np.where(w < sparse_thr, 0.0, w)
                 out[b, j, h] = w @ v[b, kv, :n]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# V sub-family v3: outlier-channel separation ([llama-tq], K-cache and V
+# sub-family sections: "v3 with outlier-channel separation", the high-quality
+# tier).  The pages name the technique only.  Reading taken: every kv-head
+# has a fixed set of k outlier channels (dimensions of the head vector),
+# chosen by calibration as the k channels of largest mean square over sample
+# vectors; their values are stored exactly as fp16 beside the codes, and the
+# vector with those channels set to zero is encoded as v1 (norm of the
+# remainder, rotation, quantisation, packing).  Reconstruction is the v1
+# reconstruction of the remainder with the outlier channels replaced by
+# their stored values, so k = 0 is v1 and k = D keeps the whole vector.
+# ---------------------------------------------------------------------------
+
+
+def outlier_channels(x: np.ndarray, k: int) -> np.ndarray:
+    """The k channels of largest mean square over the sample vectors
+    x[..., D] of one kv-head, in ascending channel order (a tie goes to the
+    lower channel index)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ms = np.mean(x.reshape(-1, d) ** 2, axis=0)
+    order = sorted(range(d), key=lambda c: (-ms[c], c))
+    return np.array(sorted(order[:k]), dtype=np.int64)
+
+
+def encode_v3(x: np.ndarray, signs: np.ndarray, bits: int, boundaries_f32: np.ndarray,
+              channels: np.ndarray):
+    """v3 encoding of the vectors x[..., D] (one kv-head) with outlier
+    channels `channels` [k].  Returns (codes, norms, values fp16 [..., k], u)."""
+    x = np.asarray(x, dtype=np.float64)
+    ch = np.asarray(channels, dtype=np.int64)
+    vals = x[..., ch].astype(np.float16)
+    rest = x.copy()
+    rest[..., ch] = 0.0
+    codes, norms, u = encode(rest, signs, bits, boundaries_f32)
+    return codes, norms, vals, u
+
+
+def dequantize_v3(codes, norms_f16, bits, centroids_f32, signs, values_f16, channels):
+    """v1 reconstruction of the remainder, outlier channels replaced by their
+    stored fp16 values."""
+    xt = dequantize(codes, norms_f16, bits, centroids_f32, signs)
+    ch = np.asarray(channels, dtype=np.int64)
+    xt[..., ch] = np.asarray(values_f16, dtype=np.float16).astype(np.float64)
+    return xt
+
+
+def decode_v3_dequant(q, k_codes, k_norms, v_codes, v_norms, v_values, v_channels, seq_lens, scale,
+                      k_bits, v_bits, k_centroids, v_centroids, signs, sparse_thr=0.0):
+    """Formulation A for a v3 V cache: dequantise, then plain attention.
+    v_values [B, Hkv, S, k] fp16; v_channels [Hkv, k]."""
+    kt = dequantize(k_codes, k_norms, k_bits, k_centroids, signs)
+    vt = np.stack([dequantize_v3(v_codes[:, h], v_norms[:, h], v_bits, v_centroids, signs,
+                                 v_values[:, h], v_channels[h]) for h in range(v_codes.shape[1])], axis=1)
+    return attention(q, kt, vt, seq_lens, scale, sparse_thr)
+
+
+def decode_v3_rotated(q, k_codes, k_norms, v_codes, v_norms, v_values, v_channels, seq_lens, scale,
+                      k_bits, v_bits, k_centroids, v_centroids, signs, sparse_thr=0.0):
+    """Formulation B for a v3 V cache: the rotated-domain decode of the
+    remainders (decode_rotated), then each outlier channel of the output
+    replaced by the weighted sum of its stored values, sum_t w_t val_t."""
+    out = decode_rotated(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale, k_bits, v_bits,
+                         k_centroids, v_centroids, signs, sparse_thr)
+    kt = dequantize(k_codes, k_norms, k_bits, k_centroids, signs)
+    ws = attention_weights(q, kt, seq_lens, scale)
+    group = q.shape[1] // k_codes.shape[1]
+    vv = np.asarray(v_values, dtype=np.float16).astype(np.float64)
+    for (b, h), w in ws.items():
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        if sparse_thr > 0:
+            w = np.where(w < sparse_thr, 0.0, w)
+        kv = h // group
+        out[b, h, np.asarray(v_channels[kv], dtype=np.int64)] = w @ vv[b, kv, :n]
     return out
 
 

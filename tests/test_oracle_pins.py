@@ -497,3 +497,104 @@ def test_sparse_gate_keeps_weights_at_the_threshold_and_drops_below():
     at = O.attention(q, k, v, [n], 1.0, sparse_thr=lo)      # w == thr is kept
     np.testing.assert_allclose(at, O.attention(q, k, v, [n], 1.0), rtol=1e-12, atol=1e-13)
     assert np.all(O.attention(q, k, v, [n], 1.0, sparse_thr=2 * hi) == 0.0)
+
+
+# ------------------------------------------------- V v3: outlier channels ---
+
+def _outlier_rows(rng, n, d=128, planted=(5, 40, 77), gain=20.0):
+    x = rng.standard_normal((n, d))
+    x[:, list(planted)] *= gain
+    return x
+
+
+def test_v3_calibration_finds_planted_channels():
+    rng = np.random.default_rng(40)
+    x = _outlier_rows(rng, 500)
+    assert list(O.outlier_channels(x, 3)) == [5, 40, 77]
+    # ties go to the lower channel: all-equal mean squares pick 0..k-1
+    assert list(O.outlier_channels(np.ones((4, 128)), 2)) == [0, 1]
+
+
+def test_v3_with_no_channel_is_v1():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((6, 256))
+    s = O.sign_vector(3)
+    c, t = O.codebook_f32(3)
+    codes, norms, vals, _ = O.encode_v3(x, s, 3, t, np.array([], dtype=np.int64))
+    c1, n1, _ = O.encode(x, s, 3, t)
+    assert np.array_equal(codes, c1) and np.array_equal(norms.view(np.uint16), n1.view(np.uint16))
+    assert vals.shape == (6, 0)
+    np.testing.assert_array_equal(O.dequantize_v3(codes, norms, 3, c, s, vals, []),
+                                  O.dequantize(c1, n1, 3, c, s))
+
+
+def test_v3_with_every_channel_is_exact_and_kept_channels_are_fp16():
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((5, 128)) * 3
+    s = O.sign_vector(0)
+    c, t = O.codebook_f32(2)
+    allc = np.arange(128)
+    codes, norms, vals, _ = O.encode_v3(x, s, 2, t, allc)
+    assert np.all(norms == 0)  # nothing is left to quantise
+    got = O.dequantize_v3(codes, norms, 2, c, s, vals, allc)
+    np.testing.assert_array_equal(got, x.astype(np.float16).astype(np.float64))
+    ch = np.array([3, 64, 100])
+    codes, norms, vals, _ = O.encode_v3(x, s, 2, t, ch)
+    got = O.dequantize_v3(codes, norms, 2, c, s, vals, ch)
+    np.testing.assert_array_equal(got[:, ch], x[:, ch].astype(np.float16).astype(np.float64))
+    # the stored norm is the remainder's
+    rest = x.copy()
+    rest[:, ch] = 0
+    np.testing.assert_array_equal(norms, np.sqrt(np.sum(rest ** 2, axis=1)).astype(np.float16)[:, None])
+
+
+def test_v3_recovers_the_snr_lost_to_outlier_channels():
+    """On vectors with three channels scaled x20, keeping them restores the
+    reconstruction SNR of plain Gaussian vectors (the remainder is Gaussian
+    again), while v1 loses most of it to the inflated block norm."""
+    rng = np.random.default_rng(43)
+    x = _outlier_rows(rng, 400)
+    s = O.sign_vector(0)
+    c, t = O.codebook_f32(3)
+    snr = lambda a, b: 10 * np.log10(np.sum(b ** 2) / np.sum((a - b) ** 2))
+    ch = O.outlier_channels(x, 3)
+    codes, norms, vals, _ = O.encode_v3(x, s, 3, t, ch)
+    v3 = O.dequantize_v3(codes, norms, 3, c, s, vals, ch)
+    c1, n1, _ = O.encode(x, s, 3, t)
+    v1 = O.dequantize(c1, n1, 3, c, s)
+    rest = x.copy()
+    rest[:, ch] = 0
+    assert snr(v3, x) > snr(v1, x) + 10
+    # the v3 error is v1's error on the remainder, outside the kept channels
+    cr, nr, _ = O.encode(rest, s, 3, t)
+    er = O.dequantize(cr, nr, 3, c, s) - rest
+    er[:, ch] = 0
+    np.testing.assert_allclose(v3 - x, er, rtol=0, atol=1e-12)
+
+
+def test_v3_decode_formulations_agree():
+    rng = np.random.default_rng(44)
+    B, H, S, D = 2, 2, 30, 256
+    s = O.sign_vector(0)
+    ck, tk = O.codebook_f32(3)
+    cv, tv = O.codebook_f32(2)
+    k = rng.standard_normal((B, H, S, D))
+    v = rng.standard_normal((B, H, S, D))
+    v[..., [7, 130, 200]] *= 15
+    kc, kn, _ = O.encode(k, s, 3, tk)
+    chans = np.stack([O.outlier_channels(v[:, h], 4) for h in range(H)])
+    enc = [O.encode_v3(v[:, h], s, 2, tv, chans[h]) for h in range(H)]
+    vc = np.stack([e[0] for e in enc], axis=1)
+    vn = np.stack([e[1] for e in enc], axis=1)
+    vv = np.stack([e[2] for e in enc], axis=1)
+    q = rng.standard_normal((B, 6, D))
+    lens = [30, 11]
+    for thr in (0.0, 0.02):
+        a = O.decode_v3_dequant(q, kc, kn, vc, vn, vv, chans, lens, 1 / 16, 3, 2, ck, cv, s, thr)
+        b = O.decode_v3_rotated(q, kc, kn, vc, vn, vv, chans, lens, 1 / 16, 3, 2, ck, cv, s, thr)
+        assert np.max(np.abs(a - b)) <= 1e-10 * np.max(np.abs(a))
+    # the outlier channels of the output are the weighted sums of the kept values
+    kt = O.dequantize(kc, kn, 3, ck, s)
+    w = O.attention_weights(q, kt, lens, 1 / 16)[(1, 5)]
+    got = O.decode_v3_rotated(q, kc, kn, vc, vn, vv, chans, lens, 1 / 16, 3, 2, ck, cv, s)[1, 5, chans[1]]
+    np.testing.assert_allclose(got, w @ vv[1, 1, :11].astype(np.float64), rtol=1e-12)
