@@ -39,7 +39,10 @@ Readings taken where the pages are silent:
     the threshold contribute zero and the rest are not renormalised;
   * V v3 (outlier-channel separation): a fixed set of k channels per kv-head
     (largest mean square on calibration vectors) kept exactly as fp16, the
-    rest of the vector encoded as v1 (see encode_v3).
+    rest of the vector encoded as v1 (see encode_v3);
+  * V v2 (group-Viterbi trellis): trellis-coded quantisation of the rotated
+    block, 4-state trellis, one 128-coordinate block per group (see
+    encode_v2).
 """
 from __future__ import annotations
 
@@ -498,3 +501,200 @@ def sparse_skip_fraction(q, k, seq_lens, scale, thr, group):
             skipped += int(np.sum(w < thr))
             total += n
     return skipped / max(total, 1)
+
+
+# ---------------------------------------------------------------------------
+# V sub-family v2: group-Viterbi trellis coding ([llama-tq], V sub-family
+# section: "v2 based on a group-Viterbi trellis", the default V format; V is
+# heavy-tailed and a trellis spends its bits where the values are).  The pages
+# name the technique only.  Reading taken: trellis-coded quantisation (TCQ,
+# Marcellin and Fischer, IEEE Trans. Commun. 38(1), 1990) of the same
+# normalised rotated coordinates u that v1 quantises, with
+#   * the doubled codebook: the 2^(b+1)-level Lloyd-Max quantiser of N(0,1)
+#     (fp32 levels), partitioned into four subsets D_k = {levels whose index
+#     is k mod 4}, each ascending with 2^(b-1) levels;
+#   * the 4-state trellis of Ungerboeck's amplitude-modulation code that TCQ
+#     uses: state s and branch bit beta lead to state ((s & 1) << 1) | beta,
+#     and the branch carries subset TCQ_SUBSET[s][beta]; even states draw
+#     from D0 u D2, odd states from D1 u D3;
+#   * a group = one 128-coordinate block, starting in state 0, no tail
+#     condition; the encoder is the Viterbi search for the path of least
+#     squared error sum_i (u_i - level_i)^2, where each branch takes the
+#     nearest level of its subset;
+#   * per coordinate b bits: the branch bit beta_i and the index j_i of the
+#     level inside its subset (level index 4 j_i + subset);
+#   * storage per block (16 b bytes, as v1): the branch-bit plane
+#     (pack_codes of beta with 1 bit, 16 bytes), then the subset-index plane
+#     (pack_codes of j with b - 1 bits);
+#   * ties: a smaller path metric wins, then the lower predecessor state, then
+#     the lower final state; inside a subset the lower level wins.
+# Norms and rotation are those of v1; the reconstruction is the v1 one with
+# the trellis levels in place of the centroids.
+# ---------------------------------------------------------------------------
+
+TCQ_NEXT = ((0, 1), (2, 3), (0, 1), (2, 3))     # [state][branch bit] -> state
+TCQ_SUBSET = ((0, 2), (1, 3), (2, 0), (3, 1))   # [state][branch bit] -> subset k
+
+
+def tcq_levels_f32(bits: int) -> np.ndarray:
+    """The doubled codebook of a b-bit v2 code: 2^(b+1) fp32 levels."""
+    return codebook_f32(bits + 1)[0]
+
+
+def _nearest_in_subset(u: float, levels: np.ndarray, k: int):
+    """(j, squared error) of the level of subset D_k nearest to u (the lower
+    level on a tie)."""
+    best_j, best_e = 0, math.inf
+    for j in range(len(levels) // 4):
+        e = (u - float(levels[4 * j + k])) ** 2
+        if e < best_e:
+            best_j, best_e = j, e
+    return best_j, best_e
+
+
+def tcq_viterbi(u: np.ndarray, levels: np.ndarray):
+    """Viterbi search over the 4-state trellis for one group of coordinates
+    u[n], from state 0.  Returns (beta[n], j[n], squared error of the path)."""
+    u = [float(v) for v in np.asarray(u, dtype=np.float64).ravel()]
+    n = len(u)
+    metric = [0.0, math.inf, math.inf, math.inf]
+    back = []  # per step and state: (predecessor, branch bit, j)
+    for i in range(n):
+        new = [math.inf] * 4
+        step = [None] * 4
+        for s_next in range(4):
+            beta = s_next & 1
+            for pred in (s_next >> 1, (s_next >> 1) | 2):   # lower predecessor first
+                assert TCQ_NEXT[pred][beta] == s_next
+                if metric[pred] == math.inf:
+                    continue
+                j, e = _nearest_in_subset(u[i], levels, TCQ_SUBSET[pred][beta])
+                cost = metric[pred] + e
+                if cost < new[s_next]:
+                    new[s_next], step[s_next] = cost, (pred, beta, j)
+        metric = new
+        back.append(step)
+    state = min(range(4), key=lambda s: (metric[s], s))
+    total = metric[state]
+    beta = np.zeros(n, dtype=np.int64)
+    jj = np.zeros(n, dtype=np.int64)
+    for i in range(n - 1, -1, -1):
+        pred, beta[i], jj[i] = back[i][state]
+        state = pred
+    return beta, jj, total
+
+
+def tcq_reconstruct(beta: np.ndarray, j: np.ndarray, levels: np.ndarray) -> np.ndarray:
+    """Levels of a path: walk the trellis from state 0 along the branch bits."""
+    out = np.zeros(len(beta))
+    state = 0
+    for i in range(len(beta)):
+        b = int(beta[i])
+        out[i] = float(levels[4 * int(j[i]) + TCQ_SUBSET[state][b]])
+        state = TCQ_NEXT[state][b]
+    return out
+
+
+def pack_v2(beta: np.ndarray, j: np.ndarray, bits: int) -> np.ndarray:
+    """The v2 block layout: branch-bit plane (16 bytes), then the subset-index
+    plane (16 (b - 1) bytes); last axes [..., 128] -> [..., 16 b]."""
+    planes = [pack_codes(beta, 1)]
+    if bits > 1:
+        planes.append(pack_codes(j, bits - 1))
+    return np.concatenate(planes, axis=-1)
+
+
+def unpack_v2(packed: np.ndarray, bits: int):
+    """Inverse of :func:`pack_v2`: (beta[..., 128], j[..., 128])."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    beta = unpack_codes(packed[..., :16], 1)
+    if bits > 1:
+        j = unpack_codes(packed[..., 16:], bits - 1)
+    else:
+        j = np.zeros_like(beta)
+    return beta, j
+
+
+def encode_v2(x: np.ndarray, signs: np.ndarray, bits: int, levels_f32: np.ndarray):
+    """v2 encoding of x[..., D]: the v1 norm and rotation, u = y / n per block,
+    then one Viterbi search per block.  Returns (codes [..., D/128, 16 b] in
+    the v2 layout, norms fp16, u, per-block squared error of the chosen
+    path)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    nb = d // BLOCK
+    blocks = x.reshape(*x.shape[:-1], nb, BLOCK)
+    n = np.sqrt(np.sum(blocks * blocks, axis=-1))
+    y = rotate(blocks, signs)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        u = np.where(n[..., None] > 0, y / n[..., None], 0.0)
+    flat = u.reshape(-1, BLOCK)
+    beta = np.zeros(flat.shape, dtype=np.int64)
+    jj = np.zeros(flat.shape, dtype=np.int64)
+    err = np.zeros(flat.shape[0])
+    for r in range(flat.shape[0]):
+        beta[r], jj[r], err[r] = tcq_viterbi(flat[r], levels_f32)
+    beta = beta.reshape(u.shape)
+    jj = jj.reshape(u.shape)
+    return pack_v2(beta, jj, bits), n.astype(np.float16), u, err.reshape(u.shape[:-1])
+
+
+def v2_levels(codes: np.ndarray, bits: int, levels_f32: np.ndarray) -> np.ndarray:
+    """Trellis levels of every coordinate of v2-coded blocks [..., 16 b] ->
+    [..., 128] (the rotated-domain values before the norm)."""
+    beta, jj = unpack_v2(codes, bits)
+    fb = beta.reshape(-1, BLOCK)
+    fj = jj.reshape(-1, BLOCK)
+    out = np.stack([tcq_reconstruct(fb[r], fj[r], levels_f32) for r in range(fb.shape[0])])
+    return out.reshape(beta.shape)
+
+
+def dequantize_v2(codes: np.ndarray, norms_f16: np.ndarray, bits: int, levels_f32: np.ndarray,
+                  signs: np.ndarray) -> np.ndarray:
+    """x~ = (n^ / d) . diag(s) . H . level[path] per block."""
+    lv = v2_levels(codes, bits, levels_f32)
+    nhat = np.asarray(norms_f16, dtype=np.float16).astype(np.float64)
+    xt = unrotate(lv, signs) * nhat[..., None]
+    return xt.reshape(*xt.shape[:-2], xt.shape[-2] * BLOCK)
+
+
+def decode_v2_dequant(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale, k_bits, v_bits,
+                      k_centroids, v_levels_f32, signs, sparse_thr=0.0):
+    """Formulation A for a v2 V cache: dequantise, then plain attention."""
+    kt = dequantize(k_codes, k_norms, k_bits, k_centroids, signs)
+    vt = dequantize_v2(v_codes, v_norms, v_bits, v_levels_f32, signs)
+    return attention(q, kt, vt, seq_lens, scale, sparse_thr)
+
+
+def decode_v2_rotated(q, k_codes, k_norms, v_codes, v_norms, seq_lens, scale, k_bits, v_bits,
+                      k_centroids, v_levels_f32, signs, sparse_thr=0.0):
+    """Formulation B for a v2 V cache: scores in the Hadamard domain from the
+    K codes; V summed in the rotated domain from the trellis levels,
+    acc = sum_t w_t (nV_t,blk / d) level_t,blk; one inverse rotation per head."""
+    q = np.asarray(q, dtype=np.float64)
+    bsz, hq, d = q.shape
+    hkv = k_codes.shape[1]
+    group = hq // hkv
+    nb = d // BLOCK
+    qhat = rotate(q, signs).reshape(bsz, hq, nb, BLOCK)
+    ck = np.asarray(k_centroids, dtype=np.float32).astype(np.float64)[unpack_codes(k_codes, k_bits)]
+    lv = v2_levels(v_codes, v_bits, v_levels_f32)
+    nk = np.asarray(k_norms, dtype=np.float16).astype(np.float64) / BLOCK
+    nv = np.asarray(v_norms, dtype=np.float16).astype(np.float64) / BLOCK
+    h_mat = hadamard(BLOCK)
+    out = np.zeros((bsz, hq, d))
+    for b in range(bsz):
+        n = int(seq_lens[b])
+        if n == 0:
+            continue
+        for h in range(hq):
+            kv = h // group
+            dots = np.einsum("tbi,bi->tb", ck[b, kv, :n], qhat[b, h])
+            s = scale * np.sum(nk[b, kv, :n] * dots, axis=1)
+            w = np.exp(s - s.max())
+            w = w / w.sum()
+            if sparse_thr > 0:
+                w = np.where(w < sparse_thr, 0.0, w)
+            acc = np.einsum("t,tb,tbi->bi", w, nv[b, kv, :n], lv[b, kv, :n])
+            out[b, h] = ((acc @ h_mat.T) * signs).reshape(d)
+    return out
