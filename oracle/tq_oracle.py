@@ -523,9 +523,12 @@ def sparse_skip_fraction(q, k, seq_lens, scale, thr, group):
 #     nearest level of its subset;
 #   * per coordinate b bits: the branch bit beta_i and the index j_i of the
 #     level inside its subset (level index 4 j_i + subset);
-#   * storage per block (16 b bytes, as v1): the branch-bit plane
-#     (pack_codes of beta with 1 bit, 16 bytes), then the subset-index plane
-#     (pack_codes of j with b - 1 bits);
+#   * storage per block (16 b bytes, as v1): 64 fields of 2b bits, one per
+#     coordinate pair (2k, 2k+1), LSB-first in a little-endian bitstream;
+#     field k = j_2k | j_2k+1 << (b-1) | beta_2k << (2b-2) | beta_2k+1 << (2b-1),
+#     so the 2b + 2 stream bits that end with field k hold everything the
+#     levels of the pair depend on (the pair's own bits and the two branch
+#     bits before it);
 #   * ties: a smaller path metric wins, then the lower predecessor state, then
 #     the lower final state; inside a subset the lower level wins.
 # Norms and rotation are those of v1; the reconstruction is the v1 one with
@@ -596,23 +599,44 @@ def tcq_reconstruct(beta: np.ndarray, j: np.ndarray, levels: np.ndarray) -> np.n
 
 
 def pack_v2(beta: np.ndarray, j: np.ndarray, bits: int) -> np.ndarray:
-    """The v2 block layout: branch-bit plane (16 bytes), then the subset-index
-    plane (16 (b - 1) bytes); last axes [..., 128] -> [..., 16 b]."""
-    planes = [pack_codes(beta, 1)]
-    if bits > 1:
-        planes.append(pack_codes(j, bits - 1))
-    return np.concatenate(planes, axis=-1)
+    """The v2 block layout: one 2b-bit field per coordinate pair, written
+    LSB-first into a little-endian bitstream of 16 b bytes; field k holds
+    j_2k, j_2k+1 (b - 1 bits each), then beta_2k, beta_2k+1.  Last axes
+    [..., 128] -> [..., 16 b]."""
+    beta = np.asarray(beta, dtype=np.int64)
+    j = np.asarray(j, dtype=np.int64)
+    assert beta.shape[-1] == BLOCK and j.shape == beta.shape
+    fb = beta.reshape(-1, BLOCK)
+    fj = j.reshape(-1, BLOCK)
+    out = np.zeros((fb.shape[0], 16 * bits), dtype=np.uint8)
+    w = bits - 1
+    for k in range(BLOCK // 2):
+        field = fj[:, 2 * k] | (fj[:, 2 * k + 1] << w) | (fb[:, 2 * k] << (2 * w)) | (fb[:, 2 * k + 1] << (2 * w + 1))
+        for t in range(2 * bits):
+            pos = 2 * bits * k + t
+            out[:, pos // 8] |= (((field >> t) & 1) << (pos % 8)).astype(np.uint8)
+    return out.reshape(*beta.shape[:-1], 16 * bits)
 
 
 def unpack_v2(packed: np.ndarray, bits: int):
     """Inverse of :func:`pack_v2`: (beta[..., 128], j[..., 128])."""
     packed = np.asarray(packed, dtype=np.uint8)
-    beta = unpack_codes(packed[..., :16], 1)
-    if bits > 1:
-        j = unpack_codes(packed[..., 16:], bits - 1)
-    else:
-        j = np.zeros_like(beta)
-    return beta, j
+    assert packed.shape[-1] == 16 * bits
+    flat = packed.reshape(-1, 16 * bits).astype(np.int64)
+    beta = np.zeros((flat.shape[0], BLOCK), dtype=np.int64)
+    j = np.zeros((flat.shape[0], BLOCK), dtype=np.int64)
+    w = bits - 1
+    for k in range(BLOCK // 2):
+        field = np.zeros(flat.shape[0], dtype=np.int64)
+        for t in range(2 * bits):
+            pos = 2 * bits * k + t
+            field |= ((flat[:, pos // 8] >> (pos % 8)) & 1) << t
+        j[:, 2 * k] = field & ((1 << w) - 1)
+        j[:, 2 * k + 1] = (field >> w) & ((1 << w) - 1)
+        beta[:, 2 * k] = (field >> (2 * w)) & 1
+        beta[:, 2 * k + 1] = (field >> (2 * w + 1)) & 1
+    shape = packed.shape[:-1] + (BLOCK,)
+    return beta.reshape(shape), j.reshape(shape)
 
 
 def encode_v2(x: np.ndarray, signs: np.ndarray, bits: int, levels_f32: np.ndarray):

@@ -686,20 +686,34 @@ def test_v2_beats_scalar_lloyd_max_and_stays_above_the_rate_distortion_bound():
 
 
 def test_v2_pack_layout_known_patterns():
+    # b = 3: 6-bit pair fields j_a | j_b << 2 | beta_a << 4 | beta_b << 5
     beta = np.zeros(128, dtype=np.int64)
-    beta[[0, 9, 127]] = 1
     jj = np.zeros(128, dtype=np.int64)
-    jj[1] = 3
-    jj[126] = 2
+    beta[1] = 1          # field 0 bit 5 -> stream bit 5
+    jj[2] = 3            # field 1 bits 0-1 -> stream bits 6, 7
+    beta[127] = 1        # field 63 bit 5 -> stream bit 383 (last bit)
+    jj[126] = 2          # field 63 bit 1 -> stream bit 379
     p = O.pack_v2(beta, jj, 3)
     assert p.shape == (48,)
-    assert p[0] == 0x01 and p[1] == 0x02 and p[15] == 0x80 and not np.any(p[2:15])
-    # j plane: 2 bits per coordinate from byte 16: j1 = 3 at bits 2-3, j126 = 2 at bit 253
-    assert p[16] == 0x0C and p[47] == 0x20 and not np.any(p[17:47])
+    assert p[0] == 0xE0 and p[47] == 0x88 and not np.any(p[1:47])
     b2, j2 = O.unpack_v2(p, 3)
     np.testing.assert_array_equal(b2, beta)
     np.testing.assert_array_equal(j2, jj)
-    assert O.pack_v2(beta, jj * 0, 1).shape == (16,)
+    # b = 2: 4-bit fields j_a | j_b << 1 | beta_a << 2 | beta_b << 3
+    p = O.pack_v2(beta, np.minimum(jj, 1), 2)
+    assert p.shape == (32,)
+    assert p[0] == 0x08 | 0x10 and p[31] == 0x80 | 0x10 and not np.any(p[1:31])
+    # b = 1: the branch bits alone, two per field
+    p = O.pack_v2(beta, jj * 0, 1)
+    assert p.shape == (16,) and p[0] == 0x02 and p[15] == 0x80
+    # round trip on random paths
+    rng = np.random.default_rng(3)
+    for bits in (1, 2, 3, 4):
+        bb = rng.integers(0, 2, size=(5, 128))
+        j = rng.integers(0, 1 << (bits - 1), size=(5, 128))
+        b2, j2 = O.unpack_v2(O.pack_v2(bb, j, bits), bits)
+        np.testing.assert_array_equal(b2, bb)
+        np.testing.assert_array_equal(j2, j)
 
 
 def test_v2_encode_is_v1_norm_and_rotation_and_zero_block():
