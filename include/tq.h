@@ -71,6 +71,9 @@ typedef enum {
 #define TQ_DEV_INTERNAL 8u       /* internal failure: the decode kernel's
                                     shared-memory plan did not match the device
                                     (nothing was computed; outputs are invalid) */
+#define TQ_DEV_CHANNEL_RANGE 16u /* v3 outlier channel outside [0, head_dim):
+                                    that entry is stored as 0 and never written
+                                    to the output */
 
 typedef enum { TQ_F32 = 0, TQ_F16 = 1 } tq_dtype;
 
@@ -157,7 +160,7 @@ size_t tq_decode_workspace_size(const tq_kv_desc* desc, int q_heads, float spars
  * Sparse-V (sparse_thr > 0): positions with w_t < sparse_thr (w the
  * normalised weight) contribute zero and the rest are not renormalised.
  *
- * Supported: head_dim 128 or 256, an even seq_cap, batch <= 4096
+ * Supported: head_dim 128 or 256, an even seq_cap, batch <= 2048
  * (TQ_ERR_UNSUPPORTED otherwise), and any q_heads / kv_heads ratio (groups
  * above 8 run in slices of 8).
  * q: device [batch, q_heads, head_dim], q_dtype TQ_F32 or TQ_F16.
@@ -291,6 +294,124 @@ int tq_decode_attention_noalloc(const tq_kv_desc* desc, const tq_codebook* k_cb,
  * misaligned pointer and TQ_ERR_CUDA if the copy fails.
  */
 int tq_read_device_status(const uint32_t* dev_status, uint32_t* bits_out, void* stream);
+
+/*
+ * V v3: outlier-channel separation ("llama-tq" article, V sub-families: "v3
+ * with outlier-channel separation", the high-quality tier; the pages name the
+ * technique only).  Reading taken here: every kv-head has a fixed set of k
+ * outlier channels (dimensions of the V vector), chosen by calibration as the
+ * k channels of largest mean square; their values are stored exactly as fp16
+ * beside the codes, and the V vector with those channels set to zero is
+ * encoded as usual (norm of the remainder, signs, WHT, codebook, packing).
+ * Decode uses the usual reconstruction of the remainder with the outlier
+ * channels replaced by their stored values; k = 0 is the plain format.  K
+ * is unchanged.
+ *
+ *   k:        0..TQ_MAX_OUTLIERS outlier channels per kv-head.
+ *   channels: device int32 [kv_heads, k], each row ascending and distinct,
+ *             values in [0, head_dim) (an entry outside it sets
+ *             TQ_DEV_CHANNEL_RANGE and is ignored).
+ *   values:   device fp16 (uint16) [batch, kv_heads, seq_cap, kp], with
+ *             kp = 8 when k <= 8 and 16 otherwise (16-byte rows); entry j of a
+ *             row holds V[channels[h][j]] and entries k..kp-1 are written 0.
+ *             16-byte aligned.
+ */
+#define TQ_MAX_OUTLIERS 16
+typedef struct {
+  int32_t k;
+  const int32_t* channels;
+  uint16_t* values;
+} tq_v_outliers;
+
+/*
+ * tq_pick_outlier_channels -- calibration of the v3 outlier channels: for
+ * every kv-head, the k channels of largest mean square over the rows of v
+ * (device [batch, kv_heads, rows, head_dim], v_dtype TQ_F32 or TQ_F16,
+ * 16-byte aligned), written ascending to `channels` (device int32
+ * [kv_heads, k]); a tie goes to the lower channel.  Asynchronous on `stream`.
+ * Returns TQ_ERR_INVALID_ARG for bad pointers or sizes (rows < 1, k outside
+ * 1..TQ_MAX_OUTLIERS or above head_dim), TQ_ERR_UNSUPPORTED for a head_dim
+ * the decode does not build (above 256), TQ_ERR_CUDA on a launch failure.
+ */
+int tq_pick_outlier_channels(const tq_kv_desc* desc, const void* v, int v_dtype, int rows, int k,
+                             int32_t* channels, void* stream);
+
+/*
+ * tq_encode_kv_v3 -- tq_encode_kv with the V side in v3 format: V rows are
+ * encoded with the channels of `vo` zeroed and their values written to
+ * vo->values (see above).  vo may be NULL or have k = 0 (then this is
+ * tq_encode_kv).  Every other argument, limit and error is that of
+ * tq_encode_kv; TQ_ERR_INVALID_ARG also for a bad vo (k out of range, null
+ * or misaligned channels / values when k > 0, or v NULL with k > 0).
+ */
+int tq_encode_kv_v3(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                    const void* k, const void* v, int in_dtype, int seq_new,
+                    const int32_t* start_pos, uint8_t* k_codes, uint16_t* k_norms,
+                    uint8_t* v_codes, uint16_t* v_norms, const tq_v_outliers* vo,
+                    uint32_t* dev_status, void* stream);
+
+/*
+ * tq_decode_attention_v3 -- tq_decode_attention over a cache whose V side is
+ * in v3 format: the output is that of the plain decode with every outlier
+ * channel c of each head replaced by sum_t w_t values[t][j] (c =
+ * channels[kv-head][j], w the softmax weights, sparse-V gated the same way).
+ * vo may be NULL or have k = 0 (then this is tq_decode_attention).  The
+ * workspace is tq_decode_workspace_size's.  Every other argument, limit and
+ * error is that of tq_decode_attention; in addition, head_dim 256 with
+ * k_bits + v_bits >= 7 returns TQ_ERR_UNSUPPORTED (a tile's codes and
+ * outlier values no longer fit the kernel's shared-memory rings).
+ */
+int tq_decode_attention_v3(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                           int q_heads, const void* q, int q_dtype, const uint8_t* k_codes,
+                           const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
+                           const tq_v_outliers* vo, const int32_t* seq_lens, float scale,
+                           float sparse_thr, float* out, void* workspace, size_t workspace_bytes,
+                           uint32_t* dev_status, void* stream);
+
+/*
+ * V v2: trellis-coded quantisation ("llama-tq" article, V sub-families: "v2
+ * based on a group Viterbi trellis", the default V format; the page names
+ * the technique only).  Reading taken here: TCQ (Marcellin and Fischer 1990)
+ * of the same normalised rotated block coordinates u that the plain format
+ * quantises.  The doubled codebook (the 2^(v_bits+1)-level Lloyd-Max
+ * quantiser of N(0,1), i.e. tq_make_codebook(v_bits + 1)) is split into four
+ * subsets D_k = {levels of index k mod 4}.  A 4-state trellis: branch bit
+ * beta moves state s to ((s & 1) << 1) | beta and draws from subset
+ * (s & 1) + 2 (beta xor (s >> 1)).  Each 128-coordinate block is one group
+ * that starts in state 0; the encoder's Viterbi search picks the path of
+ * least squared error (each branch taking the nearest level of its subset;
+ * ties to the lower predecessor state, the lower final state and the lower
+ * level).  Per coordinate v_bits bits: beta and the level's index j in its
+ * subset.  Block layout (16 * v_bits bytes, as the plain format): 64 fields
+ * of 2 * v_bits bits, LSB-first; field k = j_2k | j_2k+1 << (b-1) |
+ * beta_2k << (2b-2) | beta_2k+1 << (2b-1).  Norms and rotation are the plain
+ * format's.  Rates v_bits = 2 and 3; K is the plain format.
+ */
+
+/*
+ * tq_encode_kv_v2 -- tq_encode_kv with the V side in v2 format.  v_tcq is
+ * the doubled codebook (bits = v_bits + 1).  Every other argument, limit and
+ * error is that of tq_encode_kv; TQ_ERR_UNSUPPORTED for v_bits outside
+ * {2, 3}.  K (when given) is encoded by the plain encoder first.
+ */
+int tq_encode_kv_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_tcq,
+                    const void* k, const void* v, int in_dtype, int seq_new, const int32_t* start_pos,
+                    uint8_t* k_codes, uint16_t* k_norms, uint8_t* v_codes, uint16_t* v_norms,
+                    uint32_t* dev_status, void* stream);
+
+/*
+ * tq_decode_attention_v2 -- tq_decode_attention over a cache whose V side is
+ * in v2 format (v_tcq: the doubled codebook).  The V sum runs in the rotated
+ * domain on the trellis levels of each coordinate (a level depends on the
+ * coordinate's own code and the two branch bits before it).  Every other
+ * argument, limit and error is that of tq_decode_attention; TQ_ERR_UNSUPPORTED
+ * for v_bits outside {2, 3}.
+ */
+int tq_decode_attention_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_tcq,
+                           int q_heads, const void* q, int q_dtype, const uint8_t* k_codes,
+                           const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
+                           const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                           void* workspace, size_t workspace_bytes, uint32_t* dev_status, void* stream);
 
 /* Static description of a status code. */
 const char* tq_status_string(int status);

@@ -11,7 +11,8 @@ LIB_PATH = os.environ.get("TQ_LIBRARY") or os.path.join(_HERE, "libtq_b200.so")
 (TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_DEVICE_BOUNDS,
  TQ_ERR_SCRATCH_LIMIT) = range(7)
 TQ_NOALLOC_SCRATCH_BYTES = 64 << 20
-TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE, TQ_DEV_INTERNAL = 1, 2, 4, 8
+TQ_DEV_POS_RANGE, TQ_DEV_NORM_OVERFLOW, TQ_DEV_LEN_RANGE, TQ_DEV_INTERNAL, TQ_DEV_CHANNEL_RANGE = 1, 2, 4, 8, 16
+TQ_MAX_OUTLIERS = 16
 TQ_F32, TQ_F16 = 0, 1
 TQ_MAX_QUERY_TOKENS = 16
 
@@ -30,6 +31,10 @@ class KVDesc(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("seq_cap", ctypes.c_int32),
                 ("sign_seed", ctypes.c_uint64),
                 ("k_bits", ctypes.c_int32), ("v_bits", ctypes.c_int32)]
+
+
+class VOutliers(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int32), ("channels", c_void_p), ("values", c_void_p)]
 
 
 _P = ctypes.POINTER
@@ -53,6 +58,18 @@ SIGNATURES = {
                                             c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_float, c_float, c_void_p, c_void_p, c_void_p]),
     "tq_read_device_status": (c_int, [c_void_p, c_void_p, c_void_p]),
+    "tq_pick_outlier_channels": (c_int, [_P(KVDesc), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "tq_encode_kv_v3": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_void_p, c_void_p, c_int, c_int,
+                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, _P(VOutliers), c_void_p,
+                                c_void_p]),
+    "tq_encode_kv_v2": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_void_p, c_void_p, c_int, c_int,
+                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "tq_decode_attention_v2": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
+                                       c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "tq_decode_attention_v3": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, _P(VOutliers), c_void_p,
+                                       c_float, c_float, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "tq_status_string": (ctypes.c_char_p, [c_int]),
 }
 

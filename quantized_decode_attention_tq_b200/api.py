@@ -11,6 +11,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
+from ._lib import VOutliers as VOutliers_c
 from ._lib import (TQ_ERR_DEVICE_BOUNDS, TQ_F16, TQ_F32, TQ_OK, Codebook, KVDesc, TQError, check,
                    lib)
 
@@ -205,3 +206,120 @@ def read_device_status(status, stream=None) -> int:
     if st not in (TQ_OK, TQ_ERR_DEVICE_BOUNDS):
         raise TQError("tq_read_device_status", st)
     return int(bits.value)
+
+
+# ---- V v3: outlier-channel separation -------------------------------------
+
+@dataclass
+class VOutliers:
+    """v3 side data of one layer: channels int32 [Hkv, k] (ascending) and the
+    stored fp16 values [B, Hkv, seq_cap, kp] in an int16 tensor, kp = 8 for
+    k <= 8 else 16."""
+    k: int
+    channels: "object"
+    values: "object"
+
+    def c_struct(self) -> VOutliers_c:
+        return VOutliers_c(self.k, _ptr(self.channels, "channels"), _ptr(self.values, "values"))
+
+
+def outlier_row(k: int) -> int:
+    return 8 if k <= 8 else 16
+
+
+def alloc_outliers(desc: KVDesc, channels) -> VOutliers:
+    """VOutliers for `channels` (device int32 [Hkv, k]) with zeroed values."""
+    import torch
+    k = int(channels.shape[1])
+    values = torch.zeros((desc.batch, desc.kv_heads, desc.seq_cap, outlier_row(k)), dtype=torch.int16,
+                         device=channels.device)
+    return VOutliers(k, channels, values)
+
+
+def pick_outlier_channels(desc: KVDesc, v, k: int, stream=None):
+    """The k channels of largest mean square per kv-head over v [B, Hkv, rows, D]
+    (tq_pick_outlier_channels): device int32 [Hkv, k], ascending."""
+    import torch
+    ch = torch.empty((desc.kv_heads, k), dtype=torch.int32, device=v.device)
+    st = lib().tq_pick_outlier_channels(ctypes.byref(desc), _ptr(v, "v"), _dtype_code(v), int(v.shape[2]), k,
+                                        _ptr(ch, "channels"), _stream(stream))
+    check("tq_pick_outlier_channels", st)
+    return ch
+
+
+def encode_kv_v3(cache: Cache, k_cb: Codebook, v_cb: Codebook, vo: VOutliers, k=None, v=None, start_pos=None,
+                 status=None, stream=None) -> None:
+    """encode_kv with the V side in v3 format (tq_encode_kv_v3)."""
+    src = k if k is not None else v
+    if src is None:
+        raise ValueError("k or v is required")
+    if k is not None and v is not None and (k.shape != v.shape or k.dtype != v.dtype):
+        raise ValueError("k and v must have the same shape and dtype")
+    vs = vo.c_struct()
+    st = lib().tq_encode_kv_v3(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb),
+        _ptr(k, "k"), _ptr(v, "v"), _dtype_code(src), src.shape[2], _ptr(start_pos, "start_pos"),
+        _ptr(cache.k_codes, "k_codes") if k is not None else None,
+        _ptr(cache.k_norms, "k_norms") if k is not None else None,
+        _ptr(cache.v_codes, "v_codes") if v is not None else None,
+        _ptr(cache.v_norms, "v_norms") if v is not None else None,
+        ctypes.byref(vs), _ptr(status, "status"), _stream(stream))
+    check("tq_encode_kv_v3", st)
+
+
+def decode_attention_v3(cache: Cache, k_cb: Codebook, v_cb: Codebook, vo: VOutliers, q, seq_lens, scale: float,
+                        out, workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """decode_attention over a v3 V cache (tq_decode_attention_v3)."""
+    vs = vo.c_struct()
+    st = lib().tq_decode_attention_v3(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb), q.shape[1],
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"), ctypes.byref(vs),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention_v3", st)
+    return out
+
+
+# ---- V v2: trellis-coded quantisation --------------------------------------
+
+def make_tcq_codebook(v_bits: int) -> Codebook:
+    """The doubled codebook of the v2 format: the 2^(v_bits+1)-level Lloyd-Max
+    quantiser of N(0,1)."""
+    return make_codebook(v_bits + 1)
+
+
+def encode_kv_v2(cache: Cache, k_cb: Codebook, v_tcq: Codebook, k=None, v=None, start_pos=None, status=None,
+                 stream=None) -> None:
+    """encode_kv with the V side in v2 format (tq_encode_kv_v2)."""
+    src = k if k is not None else v
+    if src is None:
+        raise ValueError("k or v is required")
+    if k is not None and v is not None and (k.shape != v.shape or k.dtype != v.dtype):
+        raise ValueError("k and v must have the same shape and dtype")
+    st = lib().tq_encode_kv_v2(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_tcq),
+        _ptr(k, "k"), _ptr(v, "v"), _dtype_code(src), src.shape[2], _ptr(start_pos, "start_pos"),
+        _ptr(cache.k_codes, "k_codes") if k is not None else None,
+        _ptr(cache.k_norms, "k_norms") if k is not None else None,
+        _ptr(cache.v_codes, "v_codes") if v is not None else None,
+        _ptr(cache.v_norms, "v_norms") if v is not None else None,
+        _ptr(status, "status"), _stream(stream))
+    check("tq_encode_kv_v2", st)
+
+
+def decode_attention_v2(cache: Cache, k_cb: Codebook, v_tcq: Codebook, q, seq_lens, scale: float, out,
+                        workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """decode_attention over a v2 V cache (tq_decode_attention_v2)."""
+    st = lib().tq_decode_attention_v2(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_tcq), q.shape[1],
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention_v2", st)
+    return out

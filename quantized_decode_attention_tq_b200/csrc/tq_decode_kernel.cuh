@@ -178,6 +178,25 @@ __device__ __forceinline__ uint32_t addr3(const uint32_t* w, int pos, uint32_t l
   return (x & (63u << 7)) | lb;
 }
 
+// V v2 (trellis codes) pair tables: the index of pair p of a lane's window is
+// the W = 2b + 2 stream bits that end with the pair's field (the two branch
+// bits before the pair, then the field: j_a, j_b, beta_a, beta_b); entry f
+// holds half2(level a, level b) at T + f*128 + l*4, T aligned to 2^W * 128.
+template <int W>
+__device__ __forceinline__ uint32_t addr_field(const uint32_t* w, int pos, uint32_t lb) {
+  const int wi = pos >> 5, sh = pos & 31;
+  uint32_t x;
+  if (sh + W > 32) x = __funnelshift_r(w[wi], w[wi + 1], sh) << 7;
+  else x = sh >= 7 ? w[wi] >> (sh - 7) : w[wi] << (7 - sh);
+  return (x & (((1u << W) - 1u) << 7)) | lb;
+}
+template <int B>
+__device__ __forceinline__ uint2 pair2_frag_v2(const uint32_t* w, int r, uint32_t lb) {
+  static_assert(B == 2 || B == 3, "v2 rates");
+  return make_uint2(ld_table(addr_field<2 * B + 2>(w, 2 * B * (2 * r), lb)),
+                    ld_table(addr_field<2 * B + 2>(w, 2 * B * (2 * r + 1), lb)));
+}
+
 // Address of the byte-table entry indexed by the byte at bit `pos` (a
 // multiple of 8) of w, for the lane base word lbw.
 __device__ __forceinline__ uint32_t addr_byte(const uint32_t* w, int pos, uint32_t lbw) {
@@ -526,7 +545,7 @@ struct TileRegs {
 
 // Code words of one tile from a ring slot.  ks / vs are the shared addresses
 // of this lane's first K / V word in the slot.
-template <int KB, int VB, int NB, bool LOADK, bool LOADV>
+template <int KB, int VB, int NB, bool LOADK, bool LOADV, bool V2 = false>
 __device__ __forceinline__ void read_tile(TileRegs<KB, VB, NB>& r, uint32_t ks, uint32_t vs, int R) {
   if constexpr (LOADK) {
 #pragma unroll
@@ -547,13 +566,33 @@ __device__ __forceinline__ void read_tile(TileRegs<KB, VB, NB>& r, uint32_t ks, 
   }
   if constexpr (LOADV) {
     const uint32_t vsh = (VB == 3 && (R & 1)) ? 16u : 0u;
+    (void)vsh;
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk) {
         const int toff = ((tt & 1) << 1) + (tt >> 1);  // vtok(g, tt) - 4g
         const uint32_t s = vs + (toff * NB + blk) * Fmt<VB>::kBlockBytes;
-        if constexpr (VB == 4) {
+        if constexpr (V2) {
+          // v2: the lane's fields (bits [16b R, 16b R + 16b) of the block's
+          // stream) and the two bits before them (zero before the block)
+          if constexpr (VB == 3) {
+            const uint32_t w0 = ld_s32(s), w1 = ld_s32(s + 4);
+            if (R & 1) {  // the window starts at bit 14 of w0
+              r.v[tt][blk][0] = __funnelshift_r(w0, w1, 14);
+              r.v[tt][blk][1] = w1 >> 14;
+            } else {
+              const uint32_t pw = R > 0 ? ld_s32(s - 4) : 0u;
+              r.v[tt][blk][0] = __funnelshift_r(pw, w0, 30);
+              r.v[tt][blk][1] = __funnelshift_r(w0, w1, 30);
+            }
+          } else {
+            const uint32_t w0 = ld_s32(s);
+            const uint32_t pw = R > 0 ? ld_s32(s - 4) : 0u;
+            r.v[tt][blk][0] = __funnelshift_r(pw, w0, 30);
+            r.v[tt][blk][1] = w0 >> 30;
+          }
+        } else if constexpr (VB == 4) {
           const uint2 x = ld_s64(s);
           r.v[tt][blk][0] = x.x; r.v[tt][blk][1] = x.y;
         } else if constexpr (VB == 3) {
@@ -611,17 +650,23 @@ struct Misc {
   static constexpr int kWl = kWm + kCWarps * kMaxGroup;      // warp l [kCWarps][8]
   static constexpr int kQexp = kWl + kCWarps * kMaxGroup;    // [8]
   static constexpr int kLse = kQexp + kMaxGroup;             // [8]
-  static constexpr int kWtot = kLse + kMaxGroup;             // [kCWarps]
+  static constexpr int kUm = kLse + kMaxGroup;               // [8]
+  static constexpr int kUl = kUm + kMaxGroup;                // [8]
+  static constexpr int kWtot = kUl + kMaxGroup;              // [kCWarps]
   static constexpr int kWords = kWtot + kCWarps;
 };
 
 // --------------------------------------------------------------- the kernel --
 
-template <int KB, int VB, int NB, int MODE, int GQ>
+template <int KB, int VB, int NB, int MODE, int GQ, bool VO, bool V2>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   constexpr int D = NB * kBlock;
+  // floats per head of a published partial: acc, then (v3) the outlier sums
+  constexpr int PD = VO ? acc_stride(D) : D;
   constexpr bool HASK = MODE != kSparseV, HASV = MODE != kScores;
+  static_assert(!VO || HASV, "v3 outliers ride with the V pass");
+  static_assert(!V2 || (HASV && !VO && (VB == 2 || VB == 3)), "v2 trellis V: rates 2 and 3");
   constexpr int KBB = Fmt<KB>::kBlockBytes, VBB = Fmt<VB>::kBlockBytes;
   // GQ == 4 (at most four query heads per unit): score columns 4..7 repeat
   // heads 0..3, and the V products use the eight MMA columns as (head, dim
@@ -653,7 +698,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   float* w_m = misc + Misc::kWm;
   float* w_l = misc + Misc::kWl;
   int* qexp = reinterpret_cast<int*>(misc + Misc::kQexp);
-  float* u_lse = misc + Misc::kLse;
+  float* u_lse = misc + Misc::kLse;  // sparse-V pass 2, per head of the unit: log2 sum_t 2^s_t,
+  float* u_m = misc + Misc::kUm;      // the maximum score M
+  float* u_l = misc + Misc::kUl;      // and 2^-7 sum_t 2^(s_t - M)
   int* wtot = reinterpret_cast<int*>(misc + Misc::kWtot);
   int* prefix = reinterpret_cast<int*>(gptr(sm.prefix));  // [B+1] tiles per batch, prefix
   const uint32_t depth = sm.depth;
@@ -663,9 +710,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   if constexpr (KB == 3) lbK = sm.lut_k + 4u * lane;
   if constexpr (KB == 4) lbK = sm.lut_k + 4u * lane;
   if constexpr (KB == 2) lbK = sm.lut_k + 8u * (lane & 15);
-  if constexpr (VB == 3) lbV = sm.lut_v + 4u * lane;
+  if constexpr (VB == 3 || V2) lbV = sm.lut_v + 4u * lane;
   if constexpr (VB == 4) lbV = sm.lut_v + 4u * lane;
-  if constexpr (VB == 2) lbV = sm.lut_v + 8u * (lane & 15);
+  if constexpr (VB == 2 && !V2) lbV = sm.lut_v + 8u * (lane & 15);
 
   // kDup B fragments: a token's weight in the low half (s' = 0, R < 4) or
   // the high half (s' = 1) of the register, zero in the other
@@ -704,11 +751,27 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       }
     }
   };
+  // v2 pair table: entry f = (beta_{-2}, beta_{-1}, j_a, j_b, beta_a, beta_b)
+  // from bit 0 up; level index 4 j + subset, subset = beta_{i-1} + 2 (beta_i
+  // xor beta_{i-2}) (the trellis of the v2 encoder); cent = doubled codebook
+  auto fill_table_v2 = [&](int bits, const float* cent, uint32_t base, int t_first, int t_count) {
+    const int t = tid - t_first;
+    const int jw = bits - 1, n = 1 << (2 * bits + 2);
+    for (int e = t; e < n * 32; e += t_count) {
+      const int f = e >> 5;
+      const int w0 = f & 1, w1 = (f >> 1) & 1;
+      const int ja = (f >> 2) & ((1 << jw) - 1), jb = (f >> (2 + jw)) & ((1 << jw) - 1);
+      const int ba = (f >> (2 + 2 * jw)) & 1, bb = (f >> (3 + 2 * jw)) & 1;
+      const int sa = w1 + 2 * (ba ^ w0), sb = ba + 2 * (bb ^ w1);
+      *reinterpret_cast<uint32_t*>(gptr(base + 4u * e)) = pack_half2(cent[4 * ja + sa], cent[4 * jb + sb]);
+    }
+  };
   auto fill_tables = [&](int t_first, int t_count) {
     if (tid < t_first || tid >= t_first + t_count) return;
     if constexpr (HASK)
       fill_table(KB, p.kcent, KB == 3 ? sm.lut_k : sm.lut_k & ~255u, KB == 3 ? 0u : (sm.lut_k & 128u), t_first, t_count);
-    if constexpr (HASV)
+    if constexpr (HASV && V2) fill_table_v2(VB, p.vcent, sm.lut_v, t_first, t_count);
+    if constexpr (HASV && !V2)
       fill_table(VB, p.vcent, VB == 3 ? sm.lut_v : sm.lut_v & ~255u, VB == 3 ? 0u : (sm.lut_v & 128u), t_first, t_count);
   };
   bool tables_ready = false;  // filled during the first segment's query preparation
@@ -795,6 +858,28 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   const bool norm_lane = kn_lane || vn_lane;
   const int nidx = lane % kNL;
   const uint32_t ndst = (kn_lane ? sm.kn_off : sm.vn_off) + 4u * (uint32_t)nidx;
+  // V v3 outlier values: a tile's run is 16 tokens x kp fp16 (kp = 8 or 16),
+  // copied as 16-byte chunks (lane l takes chunk l).  Inside each 128-byte
+  // line of the slot the chunk index is XOR-ed with the line's low two bits,
+  // so that the fragment loads (8 tokens of one parity x 4 channel pairs)
+  // fall into 32 distinct banks.
+  auto vo_swz = [](int c) { return (uint32_t)((c >> 3) * 128 + 16 * ((c & 7) ^ ((c >> 3) & 3))); };
+  const int vo_kp = VO ? p.vo_kp : 8;
+  const bool vo_lane = VO && lane < 2 * vo_kp;
+  const uint32_t vo_dst = VO ? sm.vo_off + vo_swz(lane) : 0u;
+  const int vo_tok = (lane * 8) / vo_kp;  // the token of chunk `lane`
+  // A fragment words (token parity, channel half): lane (R, g) reads channels
+  // 8 half + 2g, +1 of token 2R + parity; transposed, they become the MMA's
+  // rows (channels) by its k (tokens, in the P^T order of the V products)
+  uint32_t vo_a[4] = {0u, 0u, 0u, 0u};
+  if constexpr (VO) {
+#pragma unroll
+    for (int par = 0; par < 2; ++par)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        if (hf == 0 || vo_kp == 16)
+          vo_a[2 * par + hf] = sm.vo_off + vo_swz((2 * R + par) * vo_kp / 8 + hf) + 4u * g;
+  }
 
   // The warp's ring is used in order across all its segments: consumed tile
   // n sits in slot n % depth, kept incrementally (cslot for consumption,
@@ -867,7 +952,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
 
   // ---- D8: o = s o (H.acc) / L for one head row held by a warp (lane l
   // holds dims 4l..4l+3 of each block) ------------------------------------------
-  auto emit_row = [&](float (&v)[NB][4], float div, int b, int vh) {
+  auto emit_row = [&](float (&v)[NB][4], const float (&ov)[4], float div, int b, int vh) {
     wht_rows<NB>(v, lane);
     const uint32_t sgn = p.sign_mask[lane >> 3] >> (4 * (lane & 7));  // signs of dims 4l..4l+3
     const float inv = div > 0.0f ? 1.0f / div : 0.0f;  // div = 0: no position seen
@@ -878,6 +963,30 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         v[blk][k] *= inv;
         if ((sgn >> k) & 1u) v[blk][k] = -v[blk][k];
       }
+    }
+    if constexpr (VO) {
+      // v3: each outlier channel of the row is the weighted sum of its stored
+      // values (original domain; the weights carry 2^-7, the divisor 128 more
+      // than the plain sum of weights)
+      const int32_t* chs = p.vo_channels + (size_t)(vh / Gv) * p.vo_k;
+      const float oinv = 128.0f * inv;
+#pragma unroll
+      for (int t = 0; t < kOutlierMax; ++t) {
+        if (t < p.vo_k) {
+          const float val = __shfl_sync(0xffffffffu, ov[t & 3], t >> 2) * oinv;
+          const int ch = __ldg(chs + t);
+          if ((ch < 0 || ch >= D) && lane == 0 && p.status) atomicOr(p.status, TQ_DEV_CHANNEL_RANGE);
+          const bool own = ch >= 0 && ch < D && lane == ((ch & (kBlock - 1)) >> 2);
+#pragma unroll
+          for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (own && (ch >> 7) == blk && (ch & 3) == k) v[blk][k] = val;
+        }
+      }
+    }
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
       *reinterpret_cast<float4*>(p.out + vrow(b, vh) * D + blk * kBlock + 4 * lane) =
           make_float4(v[blk][0], v[blk][1], v[blk][2], v[blk][3]);
     }
@@ -896,6 +1005,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     const uint8_t* ksrc = kcp + 16 * lane;  // chunk `lane` of tile 0
     const uint8_t* vsrc = vcp + 16 * lane;
     const uint16_t* nsrc = (kn_lane ? knp : vnp) + 2 * nidx;  // this lane's first norm of a tile
+    const uint16_t* vop = VO ? p.vo_values + cache_row * vo_kp : nullptr;
 
     // Copy tile `tile` of this unit into this warp's next slot (one cp.async
     // group).
@@ -912,6 +1022,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         for (int r = 0; r < kRV; ++r)
           cp_async16_if(32 * r + 32 <= kCV || lane + 32 * r < kCV, sb + vdst[r], vsrc + vt + 512 * r, 16u);
         cp_async4_if(norm_lane, sb + ndst, nsrc + (size_t)t0 * NB, 4u);
+        if constexpr (VO) cp_async16_if(vo_lane, sb + vo_dst, vop + (size_t)t0 * vo_kp + 8 * lane, 16u);
       } else {
         // the last tile of a sequence: chunks and norms past the end are
         // zero-filled (a zero code and a zero norm contribute nothing)
@@ -929,6 +1040,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         }
         const int valid = max(0, min(2, nval * NB - 2 * nidx));  // fp16 norms of this piece
         cp_async4_if(norm_lane, sb + ndst, valid ? nsrc + (size_t)t0 * NB : knp, 2u * (uint32_t)valid);
+        if constexpr (VO) {
+          const bool ok = vo_tok < nval;
+          cp_async16_if(vo_lane, sb + vo_dst, ok ? vop + (size_t)t0 * vo_kp + 8 * lane : vop, ok ? 16u : 0u);
+        }
       }
       cp_async_commit();
       if (++islot == depth) islot = 0;
@@ -961,7 +1076,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     // ---- per-unit query preparation ----------------------------------------
     uint32_t qf[NB][8][2];
     float qmul[2] = {0.0f, 0.0f};
-    float lse2[2] = {0.0f, 0.0f};
+    float lse2[2] = {0.0f, 0.0f}, moff2[2] = {0.0f, 0.0f};
     if constexpr (HASK) prep_q(b, h0, Gu, qf, qmul);
     if constexpr (MODE == kSparseV) {
       if (!tables_ready) fill_tables(0, kThreads);
@@ -971,16 +1086,24 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       const Split sp1(prefix, p.batch, UB, p1_ctas);
       if (cw < Gu) {
         const float2 ML = unit_ml_warp(p.slot_ml, sp1.part_of(Su), sp1.part_of(Su + nt - 1), sp1, unit, cw, lane);
-        if (lane == 0) u_lse[cw] = ML.x + __log2f(ML.y) + kPShift;  // pass-1 l carries 2^-7
+        if (lane == 0) {
+          const bool seen = ML.x != -INFINITY && ML.y > 0.0f;  // no position visible: weights 0
+          u_lse[cw] = seen ? ML.x + __log2f(ML.y) + kPShift : INFINITY;  // pass-1 l carries 2^-7
+          u_m[cw] = seen ? ML.x : 0.0f;
+          u_l[cw] = seen ? ML.y : 0.0f;
+        }
       }
       consumer_sync();
       const int hd0 = kDup ? (2 * g) & 3 : 2 * g, hd1 = kDup ? (2 * g + 1) & 3 : 2 * g + 1;
-      // weights carry 2^-kPShift (see the fused path)
-      lse2[0] = ((hd0 < Gu) ? u_lse[hd0] : 0.0f) + kPShift;
-      lse2[1] = ((hd1 < Gu) ? u_lse[hd1] : 0.0f) + kPShift;
-      consumer_sync();  // u_lse is reused by the next segment
+      // the gate compares s - LSE with log2(thr); the kept weights are
+      // 2^(s - M - 7), as in the fused path (normal fp16 range for the
+      // largest ones), and the output is divided by 128 * u_l at the end
+      lse2[0] = (hd0 < Gu) ? u_lse[hd0] : INFINITY;
+      lse2[1] = (hd1 < Gu) ? u_lse[hd1] : INFINITY;
+      moff2[0] = ((hd0 < Gu) ? u_m[hd0] : 0.0f) + kPShift;
+      moff2[1] = ((hd1 < Gu) ? u_m[hd1] : 0.0f) + kPShift;
     }
-    const float log2_thr = (MODE == kSparseV) ? __log2f(p.sparse_thr) - kPShift : 0.0f;
+    const float log2_thr = (MODE == kSparseV) ? __log2f(p.sparse_thr) : 0.0f;
 
     // ---- warp loop over this segment's tiles ----------------------------------
     float acc[NB][kMT][4];
@@ -990,6 +1113,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[blk][mt][e] = 0.0f;
+    // v3: outlier sums, rows = channel slots R / R + 8, columns = score columns
+    float acc_o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint32_t oa[4] = {0u, 0u, 0u, 0u};  // this tile's outlier A fragments
     // Online softmax state per score column, in the unscaled domain of
     // s' = raw * nK (the score is s = s' * qmul): m_run is the running max of
     // s, moff = m_ref + kPShift the exponent offset (m_ref = 0 while no
@@ -1046,6 +1172,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     }
     const int len_full = len - p.n_q + 1;  // tiles ending here see no mask at all
 
+    auto vfrag2 = [&](const uint32_t* w, int r) -> uint2 {
+      if constexpr (V2) return pair2_frag_v2<VB>(w, r, lbV);
+      else return pair2_frag<VB>(w, r, lbV);
+    };
     auto finish = [&](TileRegs<KB, VB, NB>& tr, int tile, const Raw& raw, auto full_tag) {
       constexpr bool FULL = decltype(full_tag)::value;
       const int t0 = tile * kTile;
@@ -1112,6 +1242,10 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
                     acc[blk][mt][cc] *= alpha;
                     acc[blk][mt][2 + cc] *= alpha;
                   }
+                if constexpr (VO) {
+                  acc_o[cc] *= alpha;
+                  acc_o[2 + cc] *= alpha;
+                }
               }
               m_run[cc] = tmax;
               moff[cc] = tmax + kPShift;
@@ -1128,8 +1262,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           l_run[cc] += pR[cc] + pR8[cc];
         }
       } else {
-        // pass 2 of sparse-V: normalised weights from the stored scores (D5),
-        // times 2^-7
+        // pass 2 of sparse-V: the gate on the normalised weight 2^(s - LSE)
+        // (D5), the kept positions weighted 2^(s - M - 7)
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int hd = kDup ? (2 * g + cc) & 3 : 2 * g + cc;
@@ -1144,9 +1278,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             } else if (okR[cc]) {
               s0 = __ldcs(srow);
             }
-            const float d0 = s0 - lse2[cc], d1 = s1 - lse2[cc];
-            wR = d0 >= log2_thr ? ex2(d0) : 0.0f;
-            wR8 = d1 >= log2_thr ? ex2(d1) : 0.0f;
+            wR = s0 - lse2[cc] >= log2_thr ? ex2(s0 - moff2[cc]) : 0.0f;
+            wR8 = s1 - lse2[cc] >= log2_thr ? ex2(s1 - moff2[cc]) : 0.0f;
           }
           pR[cc] = wR;
           pR8[cc] = wR8;
@@ -1174,26 +1307,32 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
               const uint32_t pb0 = prmt(b1, 0u, selLo), pb1 = prmt(b1, 0u, selHi);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const uint2 v0 = pair2_frag<VB>(tr.v[0][blk], q, lbV);
-                const uint2 v1 = pair2_frag<VB>(tr.v[1][blk], q, lbV);
+                const uint2 v0 = vfrag2(tr.v[0][blk], q);
+                const uint2 v1 = vfrag2(tr.v[1][blk], q);
                 mma16816(acc[blk][q], v0.x, v0.y, v1.x, v1.y, pa0, pa1);
-                const uint2 v2 = pair2_frag<VB>(tr.v[2][blk], q, lbV);
-                const uint2 v3 = pair2_frag<VB>(tr.v[3][blk], q, lbV);
+                const uint2 v2 = vfrag2(tr.v[2][blk], q);
+                const uint2 v3 = vfrag2(tr.v[3][blk], q);
                 mma16816(acc[blk][q], v2.x, v2.y, v3.x, v3.y, pb0, pb1);
               }
             } else {
 #pragma unroll
               for (int m2 = 0; m2 < 4; ++m2) {
-                const uint2 x0 = pair2_frag<VB>(tr.v[0][blk], m2, lbV);
-                const uint2 x1 = pair2_frag<VB>(tr.v[1][blk], m2, lbV);
-                const uint2 x2 = pair2_frag<VB>(tr.v[2][blk], m2, lbV);
-                const uint2 x3 = pair2_frag<VB>(tr.v[3][blk], m2, lbV);
+                const uint2 x0 = vfrag2(tr.v[0][blk], m2);
+                const uint2 x1 = vfrag2(tr.v[1][blk], m2);
+                const uint2 x2 = vfrag2(tr.v[2][blk], m2);
+                const uint2 x3 = vfrag2(tr.v[3][blk], m2);
                 mma16816(acc[blk][2 * m2], prmt(x0.x, x1.x, 0x5410), prmt(x0.x, x1.x, 0x7632),
                          prmt(x2.x, x3.x, 0x5410), prmt(x2.x, x3.x, 0x7632), b0, b1);
                 mma16816(acc[blk][2 * m2 + 1], prmt(x0.y, x1.y, 0x5410), prmt(x0.y, x1.y, 0x7632),
                          prmt(x2.y, x3.y, 0x5410), prmt(x2.y, x3.y, 0x7632), b0, b1);
               }
             }
+          }
+          if constexpr (VO) {
+            // outlier channels: sum_t w_t val_t, the plain weights (no norm)
+            const uint32_t ob0 = movtrans(pack_half2(pR[0], pR[1]));
+            const uint32_t ob1 = movtrans(pack_half2(pR8[0], pR8[1]));
+            mma16816(acc_o, oa[0], oa[1], oa[2], oa[3], ob0, ob1);
           }
         }
       }
@@ -1209,9 +1348,17 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         const uint32_t sl = wring_s + cslot * slot_bytes;
         cp_async_wait_depth(depth);  // this lane's copies of tile i have landed
         __syncwarp();                // and every other lane's
-        read_tile<KB, VB, NB, HASK, HASV>(tr, sl + koff, sl + voff, R);
+        read_tile<KB, VB, NB, HASK, HASV, V2>(tr, sl + koff, sl + voff, R);
         if constexpr (HASK) read_norms<NB>(tr.kn, sl + sm.kn_off, R);
         if constexpr (HASV) read_norms<NB>(tr.vn, sl + sm.vn_off, R);
+        if constexpr (VO) {
+          oa[0] = movtrans(ld_s32(sl + vo_a[0]));
+          oa[2] = movtrans(ld_s32(sl + vo_a[2]));
+          if (vo_kp == 16) {
+            oa[1] = movtrans(ld_s32(sl + vo_a[1]));
+            oa[3] = movtrans(ld_s32(sl + vo_a[3]));
+          }
+        }
         if (++cslot == depth) cslot = 0;
         const int tile = first + i * kCWarps;
         const Raw raw = scores(tr);
@@ -1267,6 +1414,16 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
                    __float_as_uint(acc[blk][mt][3]));
           }
       }
+      if constexpr (VO) {  // outlier sums in res: [warp][head][slot]
+        if (!kDup || g < 2) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t o = sm.res + 4u * ((cw * GQ + 2 * g + cc) * kOutlierMax + R);
+            st_s32(o, __float_as_uint(acc_o[cc]));
+            st_s32(o + 32u, __float_as_uint(acc_o[2 + cc]));
+          }
+        }
+      }
     }
     consumer_sync();
 
@@ -1315,17 +1472,35 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           }
         }
       }
+      float ov[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // v3: lane i < 4 holds outlier slots 4i..4i+3
+      if constexpr (VO) {
+        if (lane < 4) {
+#pragma unroll
+          for (int w = 0; w < kCWarps; ++w) {
+            const float4 a = ld_s128f(sm.res + 4u * ((w * GQ + hd) * kOutlierMax + 4 * lane));
+            if (fw[w] != 0.0f) {
+              ov[0] = fmaf(a.x, fw[w], ov[0]);
+              ov[1] = fmaf(a.y, fw[w], ov[1]);
+              ov[2] = fmaf(a.z, fw[w], ov[2]);
+              ov[3] = fmaf(a.w, fw[w], ov[3]);
+            }
+          }
+        }
+      }
       if (whole && MODE != kScores) {
         // this CTA saw the entire unit: no partial needed
-        emit_row(v, MODE == kFused ? L * 128.0f : 1.0f, b, h0 + hd);
+        emit_row(v, ov, (MODE == kFused ? L : u_l[hd]) * 128.0f, b, h0 + hd);
       } else {
         if (lane == 0)
           *reinterpret_cast<float2*>(p.slot_ml + (slot * kMaxGroup + hd) * 2) = make_float2(M, L);
         if constexpr (HASV) {
 #pragma unroll
           for (int blk = 0; blk < NB; ++blk)
-            *reinterpret_cast<float4*>(p.slot_acc + (slot * kMaxGroup + hd) * D + blk * kBlock + 4 * lane) =
+            *reinterpret_cast<float4*>(p.slot_acc + (slot * kMaxGroup + hd) * PD + blk * kBlock + 4 * lane) =
                 make_float4(v[blk][0], v[blk][1], v[blk][2], v[blk][3]);
+          if (VO && lane < 4)
+            *reinterpret_cast<float4*>(p.slot_acc + (slot * kMaxGroup + hd) * PD + D + 4 * lane) =
+                make_float4(ov[0], ov[1], ov[2], ov[3]);
         }
         if constexpr (MODE != kScores) {
           __threadfence();  // this lane's partial before the count
@@ -1341,8 +1516,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             __threadfence();  // every other partial of head hd is visible
             const long long c_first = sp.part_of(Su), c_last = sp.part_of(Su + nt - 1);
             const float* ml_base = p.slot_ml + ((long long)unit * kMaxGroup + hd) * 2;
-            const float* acc_base = p.slot_acc + ((long long)unit * kMaxGroup + hd) * D + 4 * lane;
-            const long long ml_stride = kMaxGroup * 2, acc_stride = (long long)kMaxGroup * D;
+            const float* acc_base = p.slot_acc + ((long long)unit * kMaxGroup + hd) * PD + 4 * lane;
+            const long long ml_stride = kMaxGroup * 2, part_stride = (long long)kMaxGroup * PD;
             // pass 1: the maximum over the partials (lane j holds part c0 + j)
             float Mx = -INFINITY;
             if constexpr (MODE == kFused) {
@@ -1362,6 +1537,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
               for (int k = 0; k < 4; ++k) u[blk][k] = 0.0f;
+            float uo[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             for (long long c0 = c_first; c0 <= c_last; c0 += 32) {
               const uint32_t emp = empty_bits(sp, c0, c_last, lane);
               const long long c = c0 + lane;
@@ -1388,7 +1564,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
                 float4 a[NB];
 #pragma unroll
                 for (int blk = 0; blk < NB; ++blk)
-                  a[blk] = __ldcg(reinterpret_cast<const float4*>(acc_base + (c0 + j) * acc_stride + blk * kBlock));
+                  a[blk] = __ldcg(reinterpret_cast<const float4*>(acc_base + (c0 + j) * part_stride + blk * kBlock));
 #pragma unroll
                 for (int blk = 0; blk < NB; ++blk) {  // skipped parts may hold anything: select, not multiply
                   u[blk][0] += wj != 0.0f ? a[blk].x * wj : 0.0f;
@@ -1396,9 +1572,16 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
                   u[blk][2] += wj != 0.0f ? a[blk].z * wj : 0.0f;
                   u[blk][3] += wj != 0.0f ? a[blk].w * wj : 0.0f;
                 }
+                if (VO && lane < 4) {
+                  const float4 a4 = __ldcg(reinterpret_cast<const float4*>(acc_base + (c0 + j) * part_stride + D));
+                  uo[0] += wj != 0.0f ? a4.x * wj : 0.0f;
+                  uo[1] += wj != 0.0f ? a4.y * wj : 0.0f;
+                  uo[2] += wj != 0.0f ? a4.z * wj : 0.0f;
+                  uo[3] += wj != 0.0f ? a4.w * wj : 0.0f;
+                }
               }
             }
-            emit_row(u, MODE == kFused ? Lx * 128.0f : 1.0f, b, h0 + hd);
+            emit_row(u, uo, (MODE == kFused ? Lx : u_l[hd]) * 128.0f, b, h0 + hd);
             if (lane == 0) p.tickets[(size_t)unit * kMaxGroup + hd] = 0u;  // ready for the next launch
           }
         }
@@ -1453,20 +1636,22 @@ struct Planner {
   }
 };
 
-template <int KB, int VB, int NB, int MODE, int GQ>
+template <int KB, int VB, int NB, int MODE, int GQ, bool VO, bool V2>
 bool plan_smem(int batch, SmemPlan& s) {
   constexpr bool HASK = MODE != kSparseV, HASV = MODE != kScores;
   constexpr int D = NB * kBlock;
   const int kb = HASK ? KB : 0, vb = HASV ? VB : 0;
   // the query scratch of one unit: GQ == 4 ? 4 : 8 padded rows
-  const uint32_t res_bytes = (uint32_t)((GQ == 4 ? 4 : kMaxGroup) * QScratch<NB>::kRow * 4);
+  // (v3: also the warps' outlier sums [warp][GQ heads][kOutlierMax] at the merge)
+  uint32_t res_bytes = (uint32_t)((GQ == 4 ? 4 : kMaxGroup) * QScratch<NB>::kRow * 4);
+  if (VO && res_bytes < (uint32_t)(kCWarps * GQ * kOutlierMax * 4)) res_bytes = kCWarps * GQ * kOutlierMax * 4;
   (void)D;
   for (int depth = kMaxDepth; depth >= 2; --depth) {
     s = SmemPlan{};
     s.base = kSmemBase;
     Planner pl(kSmemBase, kSmemBase + kMaxDyn);
     // tables
-    const bool byte_k = kb == 2 || kb == 4, byte_v = vb == 2 || vb == 4;
+    const bool byte_k = kb == 2 || kb == 4, byte_v = !V2 && (vb == 2 || vb == 4);
     if (byte_k || byte_v) {
       const uint32_t region = pl.take(65536, 65536);
       if (!region) continue;
@@ -1474,7 +1659,9 @@ bool plan_smem(int batch, SmemPlan& s) {
       if (byte_v) s.lut_v = region + 128;
     }
     if (kb == 3 && !(s.lut_k = pl.take(8192, 8192))) continue;
-    if (vb == 3 && !(s.lut_v = pl.take(8192, 8192))) continue;
+    if (!V2 && vb == 3 && !(s.lut_v = pl.take(8192, 8192))) continue;
+    const uint32_t v2_tab = V2 ? (uint32_t)(128u << (2 * vb + 2)) : 0u;  // 2^(2b+2) entries x 128 B
+    if (V2 && !(s.lut_v = pl.take(v2_tab, v2_tab))) continue;
     // slot: K runs, V runs (with gaps), K norms, V norms
     uint32_t off = 0, gk[4] = {0, 0, 0, 0}, gv[4] = {0, 0, 0, 0};
     if (HASK) {
@@ -1489,6 +1676,10 @@ bool plan_smem(int batch, SmemPlan& s) {
       off = s.vc_off[3] + 4 * NB * Fmt<VB>::kBlockBytes;
     }
     off = (off + 15) / 16 * 16;
+    if (VO) {  // v3 outlier values: 16 tokens x 16 fp16 (x 8 when k <= 8)
+      s.vo_off = off;
+      off += kTile * kOutlierMax * 2;
+    }
     s.kn_off = off;
     if (HASK) off += kTile * NB * 2;
     s.vn_off = off;
@@ -1510,7 +1701,8 @@ bool plan_smem(int batch, SmemPlan& s) {
     auto upd = [&](uint32_t a, uint32_t n) { if (a && a + n > end) end = a + n; };
     if (byte_k || byte_v) upd(byte_k ? s.lut_k : s.lut_v - 128, 65536);
     if (kb == 3) upd(s.lut_k, 8192);
-    if (vb == 3) upd(s.lut_v, 8192);
+    if (!V2 && vb == 3) upd(s.lut_v, 8192);
+    if (V2) upd(s.lut_v, v2_tab);
     for (int w = 0; w < kCWarps; ++w) upd(s.ring[w], ring_bytes);
     upd(s.res, res_bytes);
     upd(s.misc, Misc::kWords * 4);
@@ -1521,11 +1713,11 @@ bool plan_smem(int batch, SmemPlan& s) {
   return false;
 }
 
-template <int KB, int VB, int NB, int MODE, int GQ>
+template <int KB, int VB, int NB, int MODE, int GQ, bool VO, bool V2 = false>
 int run(DecodeParams& p, cudaStream_t stream, int p1_ctas, int* ctas_out) {
-  if (!plan_smem<KB, VB, NB, MODE, GQ>(p.batch, p.sm)) return TQ_ERR_UNSUPPORTED;
+  if (!plan_smem<KB, VB, NB, MODE, GQ, VO, V2>(p.batch, p.sm)) return TQ_ERR_UNSUPPORTED;
   const size_t smem = p.sm.bytes;
-  auto kern = decode_kernel<KB, VB, NB, MODE, GQ>;
+  auto kern = decode_kernel<KB, VB, NB, MODE, GQ, VO, V2>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
   static int cached_sms[64] = {0};
@@ -1549,21 +1741,31 @@ int run(DecodeParams& p, cudaStream_t stream, int p1_ctas, int* ctas_out) {
   return TQ_OK;
 }
 
-template <int KB, int VB, int NB, int GQ>
+template <int KB, int VB, int NB, int GQ, bool VO, bool V2 = false>
 int dispatch_modes(DecodeParams& p, cudaStream_t stream) {
   if (p.sparse_thr > 0.0f) {
     int p1 = 0;
-    int st = run<KB, 2, NB, kScores, GQ>(p, stream, 0, &p1);
+    int st = run<KB, 2, NB, kScores, GQ, false>(p, stream, 0, &p1);
     if (st != TQ_OK) return st;
-    return run<2, VB, NB, kSparseV, GQ>(p, stream, p1, nullptr);
+    return run<2, VB, NB, kSparseV, GQ, VO, V2>(p, stream, p1, nullptr);
   }
-  return run<KB, VB, NB, kFused, GQ>(p, stream, 0, nullptr);
+  return run<KB, VB, NB, kFused, GQ, VO, V2>(p, stream, 0, nullptr);
+}
+
+template <int KB, int VB, int NB, int GQ>
+int dispatch_vo(DecodeParams& p, cudaStream_t stream) {
+  if (p.v2) {
+    if constexpr (VB == 2 || VB == 3) return dispatch_modes<KB, VB, NB, GQ, false, true>(p, stream);
+    else return TQ_ERR_UNSUPPORTED;
+  }
+  if (p.vo_k > 0) return dispatch_modes<KB, VB, NB, GQ, true>(p, stream);
+  return dispatch_modes<KB, VB, NB, GQ, false>(p, stream);
 }
 
 template <int KB, int VB, int NB>
 int dispatch_gq(DecodeParams& p, cudaStream_t stream) {
-  if (p.q_heads / p.kv_heads * p.n_q <= 4) return dispatch_modes<KB, VB, NB, 4>(p, stream);
-  return dispatch_modes<KB, VB, NB, 8>(p, stream);
+  if (p.q_heads / p.kv_heads * p.n_q <= 4) return dispatch_vo<KB, VB, NB, 4>(p, stream);
+  return dispatch_vo<KB, VB, NB, 8>(p, stream);
 }
 
 template <int KB, int VB>

@@ -51,7 +51,7 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t (&w)[2 
   }
 }
 
-template <int BITS, bool F16, int SIDE>
+template <int BITS, bool F16, int SIDE, bool OUTL>
 __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* warp_signs) {
   constexpr int L = 1 << BITS;
   constexpr int NPOS = L / 2 - 1;  // positive decision boundaries
@@ -121,6 +121,53 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
         float4 v = ok ? __ldcs(src + 4 * c + q) : make_float4(0.f, 0.f, 0.f, 0.f);
         x[4 * c + 2 * q] = make_float2(v.x, v.y);
         x[4 * c + 2 * q + 1] = make_float2(v.z, v.w);
+      }
+    }
+  }
+
+  // ---- V v3: the outlier channels of this block are zeroed before the norm
+  // and the transform (their values are stored exactly, below) -------------
+  if constexpr (OUTL) {
+    const int kvh = (int)(bh % p.kv_heads);
+    uint32_t bm[4] = {0u, 0u, 0u, 0u};  // block mask: bit i <=> channel 128 j + i
+    for (int t = 0; t < p.vo_k; ++t) {
+      const int ch = __ldg(p.vo_channels + (size_t)kvh * p.vo_k + t) - kBlock * j;
+      if (ch >= 0 && ch < kBlock) {
+        const uint32_t bit = 1u << (ch & 31);
+        const int wsel = ch >> 5;
+        bm[0] |= wsel == 0 ? bit : 0u;
+        bm[1] |= wsel == 1 ? bit : 0u;
+        bm[2] |= wsel == 2 ? bit : 0u;
+        bm[3] |= wsel == 3 ? bit : 0u;
+      }
+    }
+    // element e of the lane's chunk c is i = 16c + 8h + e: byte 2c + h of bm
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t zb = (bm[c >> 1] >> (16 * (c & 1) + 8 * h)) & 0xFFu;
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        if ((zb >> e) & 1u) x[4 * c + e / 2].x = 0.0f;
+        if ((zb >> (e + 1)) & 1u) x[4 * c + e / 2].y = 0.0f;
+      }
+    }
+    // the lane pair of the vector's first block writes the values row:
+    // entry t = V[channels[kvh][t]] for t < k, 0 up to the padded width
+    if (j == 0 && ok) {
+      const size_t row_in = (size_t)row * p.head_dim;
+      uint16_t* dst = p.vo_values + ((size_t)bh * p.seq_cap + pos) * p.vo_kp;
+      for (int t = h; t < p.vo_kp; t += 2) {
+        __half val = __float2half_rn(0.0f);
+        if (t < p.vo_k) {
+          const int ch = __ldg(p.vo_channels + (size_t)kvh * p.vo_k + t);
+          if (ch >= 0 && ch < p.head_dim) {
+            val = F16 ? static_cast<const __half*>(in)[row_in + ch]
+                      : __float2half_rn(static_cast<const float*>(in)[row_in + ch]);
+          } else if (p.status) {
+            atomicOr(p.status, TQ_DEV_CHANNEL_RANGE);
+          }
+        }
+        dst[t] = __half_as_ushort(val);
       }
     }
   }
@@ -248,14 +295,14 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
   }
 }
 
-template <int KB, int VB, bool F16>
+template <int KB, int VB, bool F16, bool OUTL>
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_constant__ EncodeParams p) {
   __shared__ __align__(16) uint32_t signs[kEncThreads / 32][64];  // per-warp fp16 sign masks
   uint32_t* ws = signs[threadIdx.x >> 5];
   if (blockIdx.y == 0) {
-    if (p.in[0]) encode_side<KB, F16, 0>(p, ws);
+    if (p.in[0]) encode_side<KB, F16, 0, false>(p, ws);
   } else {
-    if (p.in[1]) encode_side<VB, F16, 1>(p, ws);
+    if (p.in[1]) encode_side<VB, F16, 1, OUTL>(p, ws);
   }
 }
 
@@ -266,10 +313,14 @@ int launch_kb_vb(const EncodeParams& p, cudaStream_t stream) {
   const long long grid_x = (threads + kEncThreads - 1) / kEncThreads;
   if (grid_x > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
   dim3 grid((unsigned)grid_x, 2);
-  if (p.f16)
-    encode_kernel<KB, VB, true><<<grid, kEncThreads, 0, stream>>>(p);
-  else
-    encode_kernel<KB, VB, false><<<grid, kEncThreads, 0, stream>>>(p);
+  const bool outl = p.vo_k > 0 && p.in[1] != nullptr;
+  if (p.f16) {
+    if (outl) encode_kernel<KB, VB, true, true><<<grid, kEncThreads, 0, stream>>>(p);
+    else encode_kernel<KB, VB, true, false><<<grid, kEncThreads, 0, stream>>>(p);
+  } else {
+    if (outl) encode_kernel<KB, VB, false, true><<<grid, kEncThreads, 0, stream>>>(p);
+    else encode_kernel<KB, VB, false, false><<<grid, kEncThreads, 0, stream>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 

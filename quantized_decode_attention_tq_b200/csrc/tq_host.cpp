@@ -96,6 +96,17 @@ int check_codebook(const tq_codebook* cb, int bits) {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// fp16 entries per token of a v3 values row: 8 for up to 8 channels, else 16
+int outlier_row(int k) { return k <= 8 ? 8 : 16; }
+
+int check_outliers(const tq_v_outliers* vo, int head_dim) {
+  if (!vo || vo->k == 0) return TQ_OK;
+  if (vo->k < 0 || vo->k > TQ_MAX_OUTLIERS || vo->k > head_dim) return TQ_ERR_INVALID_ARG;
+  if (!vo->channels || !vo->values || !aligned(vo->channels, 4) || !aligned(vo->values, 16))
+    return TQ_ERR_INVALID_ARG;
+  return TQ_OK;
+}
+
 }  // namespace
 
 namespace tq {
@@ -113,7 +124,7 @@ DecodeWorkspace decode_workspace_layout(int batch, int kv_heads, int q_heads, in
   w.ml_off = off;
   off = align_up(off + slots * kMaxGroup * 2 * sizeof(float), 256);
   w.acc_off = off;
-  off = align_up(off + slots * kMaxGroup * (size_t)head_dim * sizeof(float), 256);
+  off = align_up(off + slots * kMaxGroup * (size_t)acc_stride(head_dim) * sizeof(float), 256);
   w.scores_off = off;
   if (sparse) off = align_up(off + (size_t)batch * q_heads * seq_cap * sizeof(float), 256);
   w.total = off;
@@ -143,7 +154,7 @@ int validate_decode(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_co
                     int q_heads, int n_q, const void* q, int q_dtype, const uint8_t* k_codes,
                     const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
                     const int32_t* seq_lens, float scale, float sparse_thr, const float* out,
-                    const uint32_t* dev_status) {
+                    const uint32_t* dev_status, int v_fmt) {
   int st = check_desc(desc);
   if (st != TQ_OK) return st;
   if (desc->batch > tq::kMaxBatch || desc->head_dim > tq::kMaxDecodeHeadDim) return TQ_ERR_UNSUPPORTED;
@@ -161,8 +172,11 @@ int validate_decode(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_co
   if (dev_status && !aligned(dev_status, 4)) return TQ_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.0f) || std::isnan(sparse_thr)) return TQ_ERR_INVALID_ARG;
   if ((st = check_codebook(k_cb, desc->k_bits)) != TQ_OK) return st;
-  if ((st = check_codebook(v_cb, desc->v_bits)) != TQ_OK) return st;
-  return TQ_OK;
+  if (v_fmt == 2) {  // v2: the doubled codebook; rates 2 and 3
+    if (desc->v_bits != 2 && desc->v_bits != 3) return TQ_ERR_UNSUPPORTED;
+    return check_codebook(v_cb, desc->v_bits + 1);
+  }
+  return check_codebook(v_cb, desc->v_bits);
 }
 
 }  // namespace tq
@@ -175,10 +189,12 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
                   const uint8_t* v_codes, const uint16_t* v_norms,
                   const int32_t* seq_lens, float scale, float sparse_thr, float* out,
                   void* workspace, size_t workspace_bytes, uint32_t* dev_status,
-                  void* stream, const StepRows* step) {
+                  void* stream, const StepRows* step, const tq_v_outliers* vo = nullptr, int v_fmt = 1) {
   int st = tq::validate_decode(desc, k_cb, v_cb, q_heads, n_q, q, q_dtype, k_codes, k_norms, v_codes,
-                               v_norms, seq_lens, scale, sparse_thr, out, dev_status);
+                               v_norms, seq_lens, scale, sparse_thr, out, dev_status, v_fmt);
   if (st != TQ_OK) return st;
+  if ((st = check_outliers(vo, desc->head_dim)) != TQ_OK) return st;
+  if (vo && vo->k > 0 && desc->head_dim > tq::kBlock && desc->k_bits + desc->v_bits >= 7) return TQ_ERR_UNSUPPORTED;
   if (step) {
     if (step->kv_dtype != TQ_F32 && step->kv_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
     if (!step->k_new || !step->v_new || !aligned(step->k_new, 16) || !aligned(step->v_new, 16))
@@ -204,10 +220,12 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
   p.slot_ml = reinterpret_cast<float*>(base + w.ml_off);
   p.slot_acc = reinterpret_cast<float*>(base + w.acc_off);
   p.scores = sparse ? reinterpret_cast<float*>(base + w.scores_off) : nullptr;
+  const int v_levels = 1 << (desc->v_bits + (v_fmt == 2 ? 1 : 0));
   for (int j = 0; j < 16; ++j) {
     p.kcent[j] = j < (1 << desc->k_bits) ? k_cb->centroids[j] : 0.0f;
-    p.vcent[j] = j < (1 << desc->v_bits) ? v_cb->centroids[j] : 0.0f;
+    p.vcent[j] = j < v_levels ? v_cb->centroids[j] : 0.0f;
   }
+  p.v2 = v_fmt == 2 ? 1 : 0;
   sign_mask(desc->sign_seed, p.sign_mask);
   p.k_bits = desc->k_bits;
   p.v_bits = desc->v_bits;
@@ -219,6 +237,12 @@ int decode_common(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_code
   p.score_mult = (float)((double)scale * 1.4426950408889634 / tq::kBlock);
   p.sparse_thr = sparse ? sparse_thr : 0.0f;
   p.n_q = n_q;
+  if (vo && vo->k > 0) {
+    p.vo_k = vo->k;
+    p.vo_kp = outlier_row(vo->k);
+    p.vo_channels = vo->channels;
+    p.vo_values = vo->values;
+  }
   if (step) {
     p.kv_new[0] = step->k_new;
     p.kv_new[1] = step->v_new;
@@ -274,8 +298,19 @@ int tq_encode_kv(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codeb
                  const void* k, const void* v, int in_dtype, int seq_new,
                  const int32_t* start_pos, uint8_t* k_codes, uint16_t* k_norms,
                  uint8_t* v_codes, uint16_t* v_norms, uint32_t* dev_status, void* stream) {
+  return tq_encode_kv_v3(desc, k_cb, v_cb, k, v, in_dtype, seq_new, start_pos, k_codes, k_norms, v_codes,
+                         v_norms, nullptr, dev_status, stream);
+}
+
+int tq_encode_kv_v3(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                    const void* k, const void* v, int in_dtype, int seq_new,
+                    const int32_t* start_pos, uint8_t* k_codes, uint16_t* k_norms,
+                    uint8_t* v_codes, uint16_t* v_norms, const tq_v_outliers* vo,
+                    uint32_t* dev_status, void* stream) {
   int st = check_desc(desc);
   if (st != TQ_OK) return st;
+  if ((st = check_outliers(vo, desc->head_dim)) != TQ_OK) return st;
+  if (vo && vo->k > 0 && !v) return TQ_ERR_INVALID_ARG;
   if (in_dtype != TQ_F32 && in_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
   if (seq_new < 0) return TQ_ERR_INVALID_ARG;
   if (!k && !v) return TQ_ERR_INVALID_ARG;
@@ -317,6 +352,12 @@ int tq_encode_kv(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codeb
   p.head_dim = desc->head_dim;
   p.seq_cap = desc->seq_cap;
   p.seq_new = seq_new;
+  if (vo && vo->k > 0) {
+    p.vo_k = vo->k;
+    p.vo_kp = outlier_row(vo->k);
+    p.vo_channels = vo->channels;
+    p.vo_values = vo->values;
+  }
   return tq::launch_encode(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -363,6 +404,85 @@ int tq_decode_step(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_cod
   return decode_common(desc, k_cb, v_cb, q_heads, 1, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
                        seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
                        &step);
+}
+
+int tq_decode_attention_v3(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_cb,
+                           int q_heads, const void* q, int q_dtype, const uint8_t* k_codes,
+                           const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
+                           const tq_v_outliers* vo, const int32_t* seq_lens, float scale,
+                           float sparse_thr, float* out, void* workspace, size_t workspace_bytes,
+                           uint32_t* dev_status, void* stream) {
+  return decode_common(desc, k_cb, v_cb, q_heads, 1, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       nullptr, vo);
+}
+
+int tq_encode_kv_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_tcq,
+                    const void* k, const void* v, int in_dtype, int seq_new, const int32_t* start_pos,
+                    uint8_t* k_codes, uint16_t* k_norms, uint8_t* v_codes, uint16_t* v_norms,
+                    uint32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != TQ_OK) return st;
+  if (desc->v_bits != 2 && desc->v_bits != 3) return TQ_ERR_UNSUPPORTED;
+  if (in_dtype != TQ_F32 && in_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+  if (seq_new < 0) return TQ_ERR_INVALID_ARG;
+  if (!k && !v) return TQ_ERR_INVALID_ARG;
+  if (k) {
+    if (!k_codes || !k_norms || !aligned(k, 16) || !aligned(k_codes, 16) || !aligned(k_norms, 4))
+      return TQ_ERR_INVALID_ARG;
+    if ((st = check_codebook(k_cb, desc->k_bits)) != TQ_OK) return st;
+  }
+  if (v) {
+    if (!v_codes || !v_norms || !aligned(v, 16) || !aligned(v_codes, 16) || !aligned(v_norms, 4))
+      return TQ_ERR_INVALID_ARG;
+    if ((st = check_codebook(v_tcq, desc->v_bits + 1)) != TQ_OK) return st;
+  }
+  if (start_pos && !aligned(start_pos, 4)) return TQ_ERR_INVALID_ARG;
+  if (dev_status && !aligned(dev_status, 4)) return TQ_ERR_INVALID_ARG;
+  if (seq_new == 0) return TQ_OK;
+  if (k) {  // the K side is the plain format
+    st = tq_encode_kv_v3(desc, k_cb, nullptr, k, nullptr, in_dtype, seq_new, start_pos, k_codes, k_norms,
+                         nullptr, nullptr, nullptr, dev_status, stream);
+    if (st != TQ_OK || !v) return st;
+  }
+  tq::EncodeParams p{};
+  p.in[1] = v;
+  p.codes[1] = v_codes;
+  p.norms[1] = v_norms;
+  p.bits[1] = desc->v_bits;
+  for (int j = 0; j < (2 << desc->v_bits); ++j) p.tcq_levels[j] = v_tcq->centroids[j];
+  p.start_pos = start_pos;
+  p.status = dev_status;
+  sign_mask(desc->sign_seed, p.sign_mask);
+  p.f16 = in_dtype == TQ_F16;
+  p.batch = desc->batch;
+  p.kv_heads = desc->kv_heads;
+  p.head_dim = desc->head_dim;
+  p.seq_cap = desc->seq_cap;
+  p.seq_new = seq_new;
+  return tq::launch_encode_v2(p, static_cast<cudaStream_t>(stream));
+}
+
+int tq_decode_attention_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_codebook* v_tcq,
+                           int q_heads, const void* q, int q_dtype, const uint8_t* k_codes,
+                           const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
+                           const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                           void* workspace, size_t workspace_bytes, uint32_t* dev_status, void* stream) {
+  return decode_common(desc, k_cb, v_tcq, q_heads, 1, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       nullptr, nullptr, 2);
+}
+
+int tq_pick_outlier_channels(const tq_kv_desc* desc, const void* v, int v_dtype, int rows, int k,
+                             int32_t* channels, void* stream) {
+  int st = check_desc(desc);
+  if (st != TQ_OK) return st;
+  if (desc->head_dim > tq::kMaxDecodeHeadDim) return TQ_ERR_UNSUPPORTED;
+  if (v_dtype != TQ_F32 && v_dtype != TQ_F16) return TQ_ERR_INVALID_ARG;
+  if (rows < 1 || k < 1 || k > TQ_MAX_OUTLIERS || k > desc->head_dim) return TQ_ERR_INVALID_ARG;
+  if (!v || !channels || !aligned(v, 16) || !aligned(channels, 4)) return TQ_ERR_INVALID_ARG;
+  return tq::launch_pick_outliers(v, v_dtype == TQ_F16, desc->batch, desc->kv_heads, rows, desc->head_dim, k,
+                                  channels, static_cast<cudaStream_t>(stream));
 }
 
 int tq_read_device_status(const uint32_t* dev_status, uint32_t* bits_out, void* stream) {

@@ -14,7 +14,7 @@ constexpr int kBlock = 128;        // elements per rotated/quantised block
 constexpr int kTile = 16;          // tokens per decode MMA tile
 constexpr int kMaxGroup = 8;       // q-heads handled together per kv-head (MMA N = 8)
 constexpr int kMaxCtas = 1024;     // upper bound on persistent decode CTAs
-constexpr int kMaxBatch = 4096;    // decode batch limit (block-wide prefix scan)
+constexpr int kMaxBatch = 2048;    // decode batch limit (the tile prefix lives in shared memory)
 constexpr int kMaxHeadDim = 512;   // encoder: up to 4 blocks per vector
 constexpr int kMaxDecodeHeadDim = 256;  // decode kernels are built for 1 or 2 blocks
 
@@ -30,9 +30,21 @@ struct EncodeParams {
   uint32_t sign_mask[4];      // bit i set <=> s_i = -1
   int f16;                    // input dtype: 1 = fp16, 0 = fp32
   int batch, kv_heads, head_dim, seq_cap, seq_new;
+  // V v3 (vo_k > 0): channels [kv_heads, vo_k] of V are zeroed before the
+  // encoding and their values written to vo_values [.., seq_cap, vo_kp]
+  const int32_t* vo_channels;
+  uint16_t* vo_values;
+  int vo_k, vo_kp;
+  // V v2: the doubled codebook's 2^(bits + 1) levels (launch_encode_v2)
+  float tcq_levels[16];
 };
 
+int launch_pick_outliers(const void* v, int f16, int batch, int kv_heads, int rows, int head_dim, int k,
+                         int32_t* channels, cudaStream_t stream);
+
 int launch_encode(const EncodeParams& p, cudaStream_t stream);
+// V side only, in the v2 trellis format (p.in[1], p.codes[1], p.norms[1], p.bits[1] in {2, 3})
+int launch_encode_v2(const EncodeParams& p, cudaStream_t stream);
 
 constexpr int kDecodeWarps = 16;   // warps of one persistent decode CTA (one CTA per SM)
 
@@ -48,6 +60,7 @@ struct SmemPlan {
   uint32_t depth, slot_bytes;     // slots per ring, bytes per slot
   uint32_t kc_off[4], vc_off[4];  // K / V codes of tokens 4j..4j+3 within a slot
   uint32_t kn_off, vn_off;        // K / V norms within a slot
+  uint32_t vo_off;                // v3 outlier values within a slot
 };
 
 // Decode launch parameters.
@@ -64,7 +77,7 @@ struct DecodeParams {
   // workspace views
   uint32_t* tickets;   // [units][kMaxGroup] tiles counted per (unit, head)
   float* slot_ml;      // [(kMaxCtas + units) * kMaxGroup * 2]
-  float* slot_acc;     // [(kMaxCtas + units) * kMaxGroup * head_dim]
+  float* slot_acc;     // [(kMaxCtas + units) * kMaxGroup * acc_stride(head_dim)]
   float* scores;       // sparse only: [B, Hq, seq_cap] (log2-domain scores)
   float kcent[16], vcent[16];
   uint32_t sign_mask[4];
@@ -81,8 +94,20 @@ struct DecodeParams {
   uint8_t* app_codes[2];
   uint16_t* app_norms[2];
   float pos_bounds[2][7];  // positive decision boundaries of K and V, ascending
+  // V v3 (vo_k > 0): outlier channels [kv_heads, vo_k] and their values
+  // [B, Hkv, seq_cap, vo_kp] fp16
+  const int32_t* vo_channels;
+  const uint16_t* vo_values;
+  int vo_k, vo_kp;
+  // V v2 (v2 != 0): V codes are trellis pair fields, vcent the doubled
+  // codebook (2^(v_bits + 1) levels)
+  int v2;
   SmemPlan sm;        // filled by the launcher
 };
+
+constexpr int kOutlierMax = 16;   // outlier channels per kv-head, at most
+// floats per head of a partial: the rotated-domain acc, then the v3 outlier sums
+__host__ __device__ constexpr int acc_stride(int head_dim) { return head_dim + kOutlierMax; }
 
 // Workspace layout shared by the size query and the launcher.
 struct DecodeWorkspace {
@@ -99,6 +124,6 @@ int validate_decode(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_co
                     int q_heads, int n_q, const void* q, int q_dtype, const uint8_t* k_codes,
                     const uint16_t* k_norms, const uint8_t* v_codes, const uint16_t* v_norms,
                     const int32_t* seq_lens, float scale, float sparse_thr, const float* out,
-                    const uint32_t* dev_status);
+                    const uint32_t* dev_status, int v_fmt = 1);
 
 }  // namespace tq

@@ -17,6 +17,11 @@ Workloads (the five configurations the method is measured on):
   ragged  decode: B4, lengths uniform in [16384, 65536], seq_cap 65536,
           Hq16/Hkv4, D256, K3/V2, fp16 N(0,1) Q/K/V, sparse-V threshold 1e-5.
 Every decode workload uses softmax scale 1/sqrt(D) and sign seed 0.
+
+``dist="outlier_v"`` gives any decode workload V with outlier channels (the
+case the v3 format is for): K ~ N(0,1); V = N(0,1) times a per-(kv-head,
+channel) LogNormal(0, 0.5) scale, round(0.05*D) channels per kv-head (chosen
+without replacement) scaled x20.
 """
 from __future__ import annotations
 
@@ -65,12 +70,13 @@ def make(name: str, seed: int = 0, batch: int | None = None, seq: int | None = N
 
     ``seq`` overrides the cache length (and the ragged range is scaled to it
     unless ``ragged`` is given explicitly).  ``dist`` overrides the K/V
-    distribution: "normal" or "outlier_t4" (the encode-only workload's
-    outlier-channel K and Student-t(4) V) at the workload's own shapes.
+    distribution: "normal", "outlier_t4" (the encode-only workload's
+    outlier-channel K and Student-t(4) V) or "outlier_v" (outlier-channel V)
+    at the workload's own shapes.
     """
     cfg = dict(WORKLOADS[name])
     if dist is not None:
-        assert dist in ("normal", "outlier_t4"), dist
+        assert dist in ("normal", "outlier_t4", "outlier_v"), dist
         cfg["dist"] = dist
     bsz = batch if batch is not None else cfg["batch"]
     seq_cap = seq if seq is not None else cfg["seq"]
@@ -88,7 +94,7 @@ def make(name: str, seed: int = 0, batch: int | None = None, seq: int | None = N
     else:
         lens = np.full(bsz, seq_cap, dtype=np.int32)
 
-    # 2. per-channel K scales (outlier workload only)
+    # 2. per-channel K scales (outlier_t4), then V scales (outlier_v)
     kscale = None
     if cfg["dist"] == "outlier_t4":
         kscale = rng.lognormal(0.0, 1.0, size=(hkv, d))
@@ -96,6 +102,13 @@ def make(name: str, seed: int = 0, batch: int | None = None, seq: int | None = N
         for h in range(hkv):
             idx = rng.choice(d, size=n_out, replace=False)
             kscale[h, idx] *= 20.0
+    vscale = None
+    if cfg["dist"] == "outlier_v":
+        vscale = rng.lognormal(0.0, 0.5, size=(hkv, d))
+        n_out = int(round(0.05 * d))
+        for h in range(hkv):
+            idx = rng.choice(d, size=n_out, replace=False)
+            vscale[h, idx] *= 20.0
 
     # 3. K, 4. V  (one batch entry at a time)
     k = np.empty((bsz, hkv, seq_cap, d), dtype=dt)
@@ -109,7 +122,10 @@ def make(name: str, seed: int = 0, batch: int | None = None, seq: int | None = N
         if cfg["dist"] == "outlier_t4":
             v[b] = rng.standard_t(4.0, size=(hkv, seq_cap, d)).astype(dt)
         else:
-            v[b] = rng.standard_normal((hkv, seq_cap, d), dtype=np.float32).astype(dt)
+            vb = rng.standard_normal((hkv, seq_cap, d), dtype=np.float32)
+            if vscale is not None:
+                vb *= vscale[:, None, :].astype(np.float32)
+            v[b] = vb.astype(dt)
 
     # 5. Q
     q = None

@@ -24,7 +24,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol():
     names = _header_functions()
-    assert len(names) == 10
+    assert len(names) == 15
     lib = tq.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -35,6 +35,7 @@ def test_struct_layouts():
     assert ctypes.sizeof(_lib.Codebook) == 4 + 16 * 4 + 15 * 4
     assert ctypes.sizeof(_lib.KVDesc) == 32
     assert _lib.KVDesc.sign_seed.offset == 16
+    assert ctypes.sizeof(_lib.VOutliers) == 24 and _lib.VOutliers.channels.offset == 8
 
 
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
@@ -134,6 +135,7 @@ def test_decode_rejects_bad_arguments_without_launch():
     # sparse mode needs the score buffer: the dense size is too small
     assert call(thr=1e-5) == _lib.TQ_ERR_WORKSPACE
     assert call(desc=tq.kv_desc(2, 2, 384, 64, 3, 2)) in (_lib.TQ_ERR_UNSUPPORTED, _lib.TQ_ERR_WORKSPACE)
+    assert call(desc=tq.kv_desc(2049, 2, 128, 64, 3, 2)) in (_lib.TQ_ERR_UNSUPPORTED, _lib.TQ_ERR_WORKSPACE)
     odd = tq.kv_desc(2, 2, 128, 63, 3, 2)
     assert lib.tq_decode_attention(ctypes.byref(odd), ctypes.byref(cb3), ctypes.byref(cb2), 8, _fake(GOOD), 1,
                                    _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), 0.1, 0.0,
@@ -240,3 +242,78 @@ def test_read_device_status_argument_errors():
     assert lib.tq_read_device_status(_fake(GOOD + 2), ctypes.byref(bits), None) == _lib.TQ_ERR_INVALID_ARG
     assert lib.tq_status_string(_lib.TQ_ERR_DEVICE_BOUNDS).decode().startswith("the device status")
     assert lib.tq_status_string(_lib.TQ_ERR_SCRATCH_LIMIT).decode().startswith("request needs")
+
+
+def _vo(k=4, ch=GOOD, val=GOOD):
+    return _lib.VOutliers(k, _fake(ch) if ch else None, _fake(val) if val else None)
+
+
+def test_v3_encode_rejects_bad_outliers_without_launch():
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+
+    def call(vo, v=GOOD):
+        return lib.tq_encode_kv_v3(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), _fake(GOOD),
+                                   _fake(v) if v else None, 1, 4, None, _fake(GOOD), _fake(GOOD),
+                                   _fake(GOOD) if v else None, _fake(GOOD) if v else None,
+                                   ctypes.byref(vo) if vo is not None else None, None, None)
+
+    assert call(_vo(k=17)) == _lib.TQ_ERR_INVALID_ARG               # above TQ_MAX_OUTLIERS
+    assert call(_vo(k=-1)) == _lib.TQ_ERR_INVALID_ARG
+    assert call(_vo(ch=0)) == _lib.TQ_ERR_INVALID_ARG               # no channel list
+    assert call(_vo(val=0)) == _lib.TQ_ERR_INVALID_ARG              # no value buffer
+    assert call(_vo(ch=GOOD + 2)) == _lib.TQ_ERR_INVALID_ARG        # misaligned channels
+    assert call(_vo(val=GOOD + 8)) == _lib.TQ_ERR_INVALID_ARG       # values rows are 16-byte
+    assert call(_vo(), v=0) == _lib.TQ_ERR_INVALID_ARG              # v3 needs the V side
+    # k = 0 is the plain format: the checks of tq_encode_kv apply (here a no-op)
+    assert lib.tq_encode_kv_v3(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), _fake(GOOD), _fake(GOOD),
+                               1, 0, None, _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                               ctypes.byref(_vo(k=0, ch=0, val=0)), None, None) == _lib.TQ_OK
+
+
+def test_v3_decode_rejects_bad_outliers_without_launch():
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2 = tq.make_codebook(3), tq.make_codebook(2)
+    need = tq.decode_workspace_size(d, 8)
+
+    def call(vo, wsb=need, hq=8):
+        return lib.tq_decode_attention_v3(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), hq,
+                                          _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                          ctypes.byref(vo), _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD),
+                                          wsb, None, None)
+
+    assert call(_vo(k=17)) == _lib.TQ_ERR_INVALID_ARG
+    assert call(_vo(ch=0)) == _lib.TQ_ERR_INVALID_ARG
+    assert call(_vo(val=GOOD + 4)) == _lib.TQ_ERR_INVALID_ARG
+    assert call(_vo(), hq=7) == _lib.TQ_ERR_INVALID_ARG             # the plain decode's checks too
+    assert call(_vo(), wsb=need - 1) == _lib.TQ_ERR_WORKSPACE
+    # head_dim 256 with 7 or 8 bits per K/V pair: no shared-memory plan
+    d256 = tq.kv_desc(2, 2, 256, 64, 4, 3)
+    assert lib.tq_decode_attention_v3(ctypes.byref(d256), ctypes.byref(tq.make_codebook(4)), ctypes.byref(cb3), 8,
+                                      _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                      ctypes.byref(_vo()), _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD),
+                                      tq.decode_workspace_size(d256, 8), None, None) == _lib.TQ_ERR_UNSUPPORTED
+
+
+def test_pick_outlier_channels_rejects_bad_arguments_without_launch():
+    lib = tq.lib()
+
+    def call(desc=tq.kv_desc(2, 2, 128, 64, 3, 2), v=GOOD, dt=1, rows=64, k=4, ch=GOOD):
+        return lib.tq_pick_outlier_channels(ctypes.byref(desc), _fake(v) if v else None, dt, rows, k,
+                                            _fake(ch) if ch else None, None)
+
+    assert call(k=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(k=17) == _lib.TQ_ERR_INVALID_ARG
+    assert call(rows=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(dt=4) == _lib.TQ_ERR_INVALID_ARG
+    assert call(v=0) == _lib.TQ_ERR_INVALID_ARG
+    assert call(v=GOOD + 2) == _lib.TQ_ERR_INVALID_ARG
+    assert call(ch=GOOD + 1) == _lib.TQ_ERR_INVALID_ARG
+    assert call(desc=tq.kv_desc(2, 2, 384, 64, 3, 2)) == _lib.TQ_ERR_UNSUPPORTED
+    assert call(desc=tq.kv_desc(2, 2, 100, 64, 3, 2)) == _lib.TQ_ERR_UNSUPPORTED
+
+
+def test_outlier_row_width():
+    assert [tq.outlier_row(k) for k in (1, 8, 9, 16)] == [8, 8, 16, 16]
