@@ -181,20 +181,22 @@ __device__ __forceinline__ uint32_t addr3(const uint32_t* w, int pos, uint32_t l
 // V v2 (trellis codes) pair tables: the index of pair p of a lane's window is
 // the W = 2b + 2 stream bits that end with the pair's field (the two branch
 // bits before the pair, then the field: j_a, j_b, beta_a, beta_b); entry f
-// holds half2(level a, level b) at T + f*128 + l*4, T aligned to 2^W * 128.
-template <int W>
+// holds half2(level a, level b) at T + (f << S) + l*4, S = 7 for a table of
+// its own (T aligned to 2^(W+7)) or S = 8 in the free V half of a byte-table
+// region (T = region + 128, the region 64 KiB-aligned).
+template <int W, int S>
 __device__ __forceinline__ uint32_t addr_field(const uint32_t* w, int pos, uint32_t lb) {
   const int wi = pos >> 5, sh = pos & 31;
   uint32_t x;
-  if (sh + W > 32) x = __funnelshift_r(w[wi], w[wi + 1], sh) << 7;
-  else x = sh >= 7 ? w[wi] >> (sh - 7) : w[wi] << (7 - sh);
-  return (x & (((1u << W) - 1u) << 7)) | lb;
+  if (sh + W > 32) x = __funnelshift_r(w[wi], w[wi + 1], sh) << S;
+  else x = sh >= S ? w[wi] >> (sh - S) : w[wi] << (S - sh);
+  return (x & (((1u << W) - 1u) << S)) | lb;
 }
-template <int B>
+template <int B, int S>
 __device__ __forceinline__ uint2 pair2_frag_v2(const uint32_t* w, int r, uint32_t lb) {
   static_assert(B == 2 || B == 3, "v2 rates");
-  return make_uint2(ld_table(addr_field<2 * B + 2>(w, 2 * B * (2 * r), lb)),
-                    ld_table(addr_field<2 * B + 2>(w, 2 * B * (2 * r + 1), lb)));
+  return make_uint2(ld_table(addr_field<2 * B + 2, S>(w, 2 * B * (2 * r), lb)),
+                    ld_table(addr_field<2 * B + 2, S>(w, 2 * B * (2 * r + 1), lb)));
 }
 
 // Address of the byte-table entry indexed by the byte at bit `pos` (a
@@ -667,6 +669,8 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   constexpr bool HASK = MODE != kSparseV, HASV = MODE != kScores;
   static_assert(!VO || HASV, "v3 outliers ride with the V pass");
   static_assert(!V2 || (HASV && !VO && (VB == 2 || VB == 3)), "v2 trellis V: rates 2 and 3");
+  // a v2 table shares the byte-table region of a 2- or 4-bit K side
+  constexpr int V2S = (V2 && HASK && (KB == 2 || KB == 4)) ? 8 : 7;
   constexpr int KBB = Fmt<KB>::kBlockBytes, VBB = Fmt<VB>::kBlockBytes;
   // GQ == 4 (at most four query heads per unit): score columns 4..7 repeat
   // heads 0..3, and the V products use the eight MMA columns as (head, dim
@@ -758,12 +762,13 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     const int t = tid - t_first;
     const int jw = bits - 1, n = 1 << (2 * bits + 2);
     for (int e = t; e < n * 32; e += t_count) {
-      const int f = e >> 5;
+      const int f = e >> 5, l = e & 31;
       const int w0 = f & 1, w1 = (f >> 1) & 1;
       const int ja = (f >> 2) & ((1 << jw) - 1), jb = (f >> (2 + jw)) & ((1 << jw) - 1);
       const int ba = (f >> (2 + 2 * jw)) & 1, bb = (f >> (3 + 2 * jw)) & 1;
       const int sa = w1 + 2 * (ba ^ w0), sb = ba + 2 * (bb ^ w1);
-      *reinterpret_cast<uint32_t*>(gptr(base + 4u * e)) = pack_half2(cent[4 * ja + sa], cent[4 * jb + sb]);
+      *reinterpret_cast<uint32_t*>(gptr(base + ((uint32_t)f << V2S) + 4u * l)) =
+          pack_half2(cent[4 * ja + sa], cent[4 * jb + sb]);
     }
   };
   auto fill_tables = [&](int t_first, int t_count) {
@@ -1173,7 +1178,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     const int len_full = len - p.n_q + 1;  // tiles ending here see no mask at all
 
     auto vfrag2 = [&](const uint32_t* w, int r) -> uint2 {
-      if constexpr (V2) return pair2_frag_v2<VB>(w, r, lbV);
+      if constexpr (V2) return pair2_frag_v2<VB, V2S>(w, r, lbV);
       else return pair2_frag<VB>(w, r, lbV);
     };
     auto finish = [&](TileRegs<KB, VB, NB>& tr, int tile, const Raw& raw, auto full_tag) {
@@ -1660,8 +1665,11 @@ bool plan_smem(int batch, SmemPlan& s) {
     }
     if (kb == 3 && !(s.lut_k = pl.take(8192, 8192))) continue;
     if (!V2 && vb == 3 && !(s.lut_v = pl.take(8192, 8192))) continue;
-    const uint32_t v2_tab = V2 ? (uint32_t)(128u << (2 * vb + 2)) : 0u;  // 2^(2b+2) entries x 128 B
-    if (V2 && !(s.lut_v = pl.take(v2_tab, v2_tab))) continue;
+    // v2: in the V half of the byte-table region, or a table of its own
+    // (2^(2b+2) entries x 128 B)
+    const uint32_t v2_tab = (V2 && !byte_k) ? (uint32_t)(128u << (2 * vb + 2)) : 0u;
+    if (V2 && byte_k) s.lut_v = s.lut_k + 128;
+    if (v2_tab && !(s.lut_v = pl.take(v2_tab, v2_tab))) continue;
     // slot: K runs, V runs (with gaps), K norms, V norms
     uint32_t off = 0, gk[4] = {0, 0, 0, 0}, gv[4] = {0, 0, 0, 0};
     if (HASK) {
@@ -1702,7 +1710,7 @@ bool plan_smem(int batch, SmemPlan& s) {
     if (byte_k || byte_v) upd(byte_k ? s.lut_k : s.lut_v - 128, 65536);
     if (kb == 3) upd(s.lut_k, 8192);
     if (!V2 && vb == 3) upd(s.lut_v, 8192);
-    if (V2) upd(s.lut_v, v2_tab);
+    if (v2_tab) upd(s.lut_v, v2_tab);
     for (int w = 0; w < kCWarps; ++w) upd(s.ring[w], ring_bytes);
     upd(s.res, res_bytes);
     upd(s.misc, Misc::kWords * 4);

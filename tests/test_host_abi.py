@@ -317,3 +317,32 @@ def test_pick_outlier_channels_rejects_bad_arguments_without_launch():
 
 def test_outlier_row_width():
     assert [tq.outlier_row(k) for k in (1, 8, 9, 16)] == [8, 8, 16, 16]
+
+
+def test_v2_entry_points_reject_bad_arguments_without_launch():
+    lib = tq.lib()
+    cb3 = tq.make_codebook(3)
+
+    def enc(desc, vtq, k=GOOD, v=GOOD, seq_new=4):
+        return lib.tq_encode_kv_v2(ctypes.byref(desc), ctypes.byref(cb3), ctypes.byref(vtq),
+                                   _fake(k) if k else None, _fake(v) if v else None, 1, seq_new, None,
+                                   _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD), None, None)
+
+    d3 = tq.kv_desc(2, 2, 128, 64, 3, 3)
+    assert enc(d3, tq.make_codebook(3)) == _lib.TQ_ERR_INVALID_ARG       # V needs the doubled codebook
+    assert enc(tq.kv_desc(2, 2, 128, 64, 3, 4), tq.make_codebook(4)) == _lib.TQ_ERR_UNSUPPORTED  # rate 4
+    assert enc(d3, tq.make_tcq_codebook(3), k=0, v=0) == _lib.TQ_ERR_INVALID_ARG
+    assert enc(d3, tq.make_tcq_codebook(3), v=GOOD + 8) == _lib.TQ_ERR_INVALID_ARG
+    assert enc(d3, tq.make_tcq_codebook(3), seq_new=0) == _lib.TQ_OK            # no-op
+
+    def dec(desc, vtq, wsb=None):
+        need = tq.decode_workspace_size(desc, 8)
+        return lib.tq_decode_attention_v2(ctypes.byref(desc), ctypes.byref(cb3), ctypes.byref(vtq), 8,
+                                          _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                          _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD),
+                                          need if wsb is None else wsb, None, None)
+
+    d2 = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    assert dec(d2, tq.make_codebook(2)) == _lib.TQ_ERR_INVALID_ARG
+    assert dec(tq.kv_desc(2, 2, 128, 64, 3, 4), tq.make_codebook(4)) == _lib.TQ_ERR_UNSUPPORTED
+    assert dec(d2, tq.make_tcq_codebook(2), wsb=16) == _lib.TQ_ERR_WORKSPACE
