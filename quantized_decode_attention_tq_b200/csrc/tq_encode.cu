@@ -15,8 +15,15 @@
 // and lane 1 chunks 8..15 (8*b bytes each, plain vector stores) after the
 // pair swaps four chunk words.  For fp16 input the random signs are applied
 // to the fp16 sign bits as the elements are converted (one XOR per pair).
+//
+// The grid is persistent (as many CTAs as fit, split between K and V); each
+// lane pair walks blocks with a grid stride and copies the next block into a
+// per-warp staging area with cp.async while it transforms the current one,
+// so the loads stay in flight through the arithmetic.
 
 #include <cuda_fp16.h>
+
+#include <algorithm>
 
 #include "../../include/tq.h"
 #include "tq_internal.h"
@@ -24,7 +31,7 @@
 namespace tq {
 namespace {
 
-constexpr int kEncThreads = 256;
+constexpr int kEncThreads = 128;
 
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
@@ -51,26 +58,68 @@ __device__ __forceinline__ void store_codes(uint8_t* dst, const uint32_t (&w)[2 
   }
 }
 
+// 16-byte chunks a lane copies per block: fp16 8, fp32 16.  Staging of one
+// warp: 2 stages x chunks x 32 lanes x 16 B, chunk c of lane l at (c * 32 + l) * 16.
+template <bool F16>
+__host__ __device__ constexpr int lane_chunks() { return F16 ? 8 : 16; }
+template <bool F16>
+__host__ __device__ constexpr uint32_t stage_bytes() { return (uint32_t)lane_chunks<F16>() * 32 * 16; }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ uint4 ld_shared16(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// The lane's chunks of block blk into staging `st` (one commit group; an
+// empty group past the end keeps the waits counting right).
+template <bool F16>
+__device__ __forceinline__ void stage_block(const EncodeParams& p, const void* in, uint32_t blk, uint32_t n_blocks,
+                                            uint32_t st, int lane) {
+  if (blk < n_blocks) {
+    const int nb = p.head_dim / kBlock;
+    const int lnb = nb == 1 ? 0 : nb == 2 ? 1 : 2;  // nb is 1, 2 or 4
+    const size_t base = (size_t)(blk >> lnb) * p.head_dim + (size_t)(blk & (nb - 1)) * kBlock + 8 * (lane & 1);
+#pragma unroll
+    for (int c = 0; c < lane_chunks<F16>(); ++c) {
+      // fp16: chunk c is elements 16c + 8h .. +7; fp32: half c & 1 of that chunk for c / 2
+      const void* src = F16 ? static_cast<const void*>(static_cast<const __half*>(in) + base + 16 * c)
+                            : static_cast<const void*>(static_cast<const float*>(in) + base + 16 * (c >> 1) + 4 * (c & 1));
+      cp_async16(st + (uint32_t)(c * 32 + lane) * 16u, src);
+    }
+  }
+  cp_async_commit();
+}
+
 template <int BITS, bool F16, int SIDE, bool OUTL>
-__device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* warp_signs) {
+__device__ __forceinline__ void encode_block(const EncodeParams& p, const uint32_t* warp_signs, uint32_t blk,
+                                             uint32_t n_blocks, uint32_t st) {
   constexpr int L = 1 << BITS;
   constexpr int NPOS = L / 2 - 1;  // positive decision boundaries
   const void* in = p.in[SIDE];
   const int lane = threadIdx.x & 31;
   const int h = lane & 1;
   const int nb = p.head_dim / kBlock;
-  const long long n_blocks = (long long)p.batch * p.kv_heads * p.seq_new * nb;
-  const long long blk = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 1;
+  // the host keeps the flattened block count below 2^31: 32-bit index math,
+  // divisions by multiply-high (a 64-bit division is a long subroutine)
   const bool valid = blk < n_blocks;
 
   int b = 0, j = 0, t = 0;
   long long row = 0, bh = 0;
   if (valid) {
-    j = (int)(blk % nb);
-    row = blk / nb;
-    t = (int)(row % p.seq_new);
-    bh = row / p.seq_new;
-    b = (int)(bh / p.kv_heads);
+    const int lnb = nb == 1 ? 0 : nb == 2 ? 1 : 2;  // nb is 1, 2 or 4
+    j = (int)(blk & (nb - 1));
+    const uint32_t r32 = blk >> lnb;
+    const uint32_t bh32 = p.div_seq_new.div(r32);
+    t = (int)(r32 - bh32 * (uint32_t)p.seq_new);
+    b = (int)p.div_kv_heads.div(bh32);
+    row = r32;
+    bh = bh32;
   }
   int pos = t;
   if (valid && p.start_pos) pos += __ldg(p.start_pos + b);
@@ -80,25 +129,11 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
   // ---- load 64 elements (E1), convert to fp32 --------------------------
   float2 x[32];
   if constexpr (F16) {
-    // chunk 2c + h of the block (8 elements, 16 B): a lane pair reads 32
-    // contiguous bytes per load
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(in) +
-                                                      (row * p.head_dim + j * kBlock)) + h;
+    // chunk 2c + h of the block (8 elements, 16 B), staged by this lane
     uint4 raw[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) raw[c] = ok ? __ldcs(src + 2 * c) : make_uint4(0, 0, 0, 0);
-    // s o x (E1) on the fp16 bits, one mask word per element pair: word m of
-    // lane half hh covers elements i, i+1 with i = 16(m/4) + 8hh + 2(m%4),
-    // s_i in bit 15 and s_(i+1) in bit 31.  Each warp builds its own copy
-    // while its loads are in flight.
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int i = 16 * (lane >> 2) + 8 * hh + 2 * (lane & 3);
-      const uint32_t wd = p.sign_mask[i >> 5];
-      const int bit = i & 31;
-      warp_signs[hh * 32 + lane] = (((wd >> bit) & 1u) << 15) | (((wd >> (bit + 1)) & 1u) << 31);
-    }
-    __syncwarp();
+    for (int c = 0; c < 8; ++c) raw[c] = valid ? ld_shared16(st + (uint32_t)(c * 32 + lane) * 16u) : make_uint4(0, 0, 0, 0);
+    // s o x (E1) on the fp16 bits (the per-warp mask words, see encode_kernel)
     const uint4* sgn = reinterpret_cast<const uint4*>(warp_signs + 32 * h);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -112,13 +147,13 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
       }
     }
   } else {
-    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(in) +
-                                                        (row * p.head_dim + j * kBlock + 8 * h));
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        float4 v = ok ? __ldcs(src + 4 * c + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const uint4 u = valid ? ld_shared16(st + (uint32_t)((2 * c + q) * 32 + lane) * 16u) : make_uint4(0, 0, 0, 0);
+        const float4 v = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z),
+                                     __uint_as_float(u.w));
         x[4 * c + 2 * q] = make_float2(v.x, v.y);
         x[4 * c + 2 * q + 1] = make_float2(v.z, v.w);
       }
@@ -236,30 +271,36 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
   for (int k = 0; k < NPOS; ++k) thr[k] = p.pos_bounds[SIDE][k] * n;
 
   // Codes of the lane's chunk c (8 codes, 8*BITS bits) in g[c]; chunk c of
-  // lane h is chunk 2c + h of the block.
+  // lane h is chunk 2c + h of the block.  With m = #{T_k < |y|/n}, the code is
+  // L/2 - 1 - m = (L/2 - 1) ^ m for y <= 0 and L/2 + m = (L/2 - 1) ^ m ^ (L - 1)
+  // for y > 0, so every field starts at L/2 - 1 and each decision bit of the
+  // bisection, and the sign, toggles bits of it in place.
+  constexpr uint32_t kNeg = (uint32_t)(L / 2 - 1) * (BITS == 2 ? 0x5555u : BITS == 3 ? 0x249249u : 0x11111111u);
   uint32_t g[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) g[c] = 0;
+  for (int c = 0; c < 8; ++c) g[c] = kNeg;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     const float y = (i & 1) ? x[i >> 1].y : x[i >> 1].x;
     const float a = fabsf(y);
-    // m = #{k : T_k < |y|/n}, found by bisection of the ascending T_k
-    int m;
+    const int sh = BITS * (i & 7);
+    uint32_t& gw = g[i >> 3];
+    // m = #{k : T_k < |y|/n}, by bisection of the ascending T_k
     if constexpr (NPOS == 1) {
-      m = (a > thr[0]) ? 1 : 0;
+      if (a > thr[0]) gw ^= 1u << sh;
     } else if constexpr (NPOS == 3) {
-      const int c1 = (a > thr[1]) ? 1 : 0;
-      m = 2 * c1 + ((a > (c1 ? thr[2] : thr[0])) ? 1 : 0);
+      const bool c1 = a > thr[1];
+      if (c1) gw ^= 2u << sh;
+      if (a > (c1 ? thr[2] : thr[0])) gw ^= 1u << sh;
     } else {
-      const int c2 = (a > thr[3]) ? 1 : 0;
-      const int c1 = (a > (c2 ? thr[5] : thr[1])) ? 1 : 0;
+      const bool c2 = a > thr[3];
+      const bool c1 = a > (c2 ? thr[5] : thr[1]);
       const float t0 = c2 ? (c1 ? thr[6] : thr[4]) : (c1 ? thr[2] : thr[0]);
-      m = 4 * c2 + 2 * c1 + ((a > t0) ? 1 : 0);
+      if (c2) gw ^= 4u << sh;
+      if (c1) gw ^= 2u << sh;
+      if (a > t0) gw ^= 1u << sh;
     }
-    const int lowside = L / 2 - 1 - m;
-    const uint32_t idx = (uint32_t)(y > 0.0f ? (lowside ^ (L - 1)) : lowside);
-    g[i >> 3] |= idx << (BITS * (i & 7));
+    if (y > 0.0f) gw ^= (uint32_t)(L - 1) << sh;
   }
   // ---- pack (E5): LSB-first bitstream.  Lane 0 stores chunks 0..7, lane 1
   // chunks 8..15; the pair swaps the four chunk words each needs.
@@ -295,33 +336,84 @@ __device__ __forceinline__ void encode_side(const EncodeParams& p, uint32_t* war
   }
 }
 
+template <int BITS, bool F16, int SIDE, bool OUTL>
+__device__ __forceinline__ void encode_side(const EncodeParams& p, const uint32_t* ws, uint32_t st0,
+                                            uint32_t n_blocks) {
+  const int lane = threadIdx.x & 31;
+  // lane pairs walk the blocks with a grid stride; the warp stays together
+  // (its pairs are consecutive) so the loop is warp-uniform
+  const uint32_t pairs = (gridDim.x * blockDim.x) >> 1;
+  const uint32_t warp0 = (blockIdx.x * blockDim.x + (threadIdx.x & ~31u)) >> 1;
+  const uint32_t mine = lane >> 1;
+  if (warp0 >= n_blocks) return;
+  stage_block<F16>(p, p.in[SIDE], warp0 + mine, n_blocks, st0, lane);
+  uint32_t s = 0;
+  for (uint32_t base = warp0; base < n_blocks; base += pairs) {
+    stage_block<F16>(p, p.in[SIDE], base + pairs + mine, n_blocks, st0 + (s ^ 1u) * stage_bytes<F16>(), lane);
+    cp_async_wait1();  // this lane's chunks of the current block have landed
+    encode_block<BITS, F16, SIDE, OUTL>(p, ws, base + mine, n_blocks, st0 + s * stage_bytes<F16>());
+    s ^= 1u;
+  }
+}
+
 template <int KB, int VB, bool F16, bool OUTL>
 __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_constant__ EncodeParams p) {
   __shared__ __align__(16) uint32_t signs[kEncThreads / 32][64];  // per-warp fp16 sign masks
-  uint32_t* ws = signs[threadIdx.x >> 5];
-  if (blockIdx.y == 0) {
-    if (p.in[0]) encode_side<KB, F16, 0, false>(p, ws);
-  } else {
-    if (p.in[1]) encode_side<VB, F16, 1, OUTL>(p, ws);
+  extern __shared__ __align__(16) uint8_t stage[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t* ws = signs[warp];
+  if constexpr (F16) {
+    // sign mask words for s o x on the fp16 bits: word m of lane half hh
+    // covers elements i, i+1 with i = 16(m/4) + 8hh + 2(m%4), s_i in bit 15
+    // and s_(i+1) in bit 31
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = 16 * (lane >> 2) + 8 * hh + 2 * (lane & 3);
+      const uint32_t wd = p.sign_mask[i >> 5];
+      const int bit = i & 31;
+      ws[hh * 32 + lane] = (((wd >> bit) & 1u) << 15) | (((wd >> (bit + 1)) & 1u) << 31);
+    }
+    __syncwarp();
   }
+  const uint32_t st0 = (uint32_t)__cvta_generic_to_shared(stage) + (uint32_t)warp * 2u * stage_bytes<F16>();
+  const uint32_t n_blocks = (uint32_t)p.batch * p.kv_heads * p.seq_new * (p.head_dim / kBlock);
+  // grid.y: both sides (y = side) or the one side present
+  const int side = gridDim.y == 2 ? (int)blockIdx.y : (p.in[0] ? 0 : 1);
+  if (side == 0) encode_side<KB, F16, 0, false>(p, ws, st0, n_blocks);
+  else encode_side<VB, F16, 1, OUTL>(p, ws, st0, n_blocks);
+}
+
+// Persistent launch: as many CTAs as are resident at once (split between the
+// sides), at most one lane pair per block.
+template <typename K>
+int launch_typed(K kern, uint32_t stage, const EncodeParams& p, long long n_blocks, int sides, cudaStream_t stream) {
+  const size_t smem = (size_t)(kEncThreads / 32) * 2 * stage;
+  int dev = 0, sms = 0, occ = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TQ_ERR_CUDA;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kEncThreads, smem) != cudaSuccess) return TQ_ERR_CUDA;
+  if (occ < 1) return TQ_ERR_UNSUPPORTED;
+  const long long per_side = std::max(1LL, (long long)occ * sms / sides);
+  const long long needed = (n_blocks * 2 + kEncThreads - 1) / kEncThreads;
+  dim3 grid((unsigned)std::min(per_side, needed), (unsigned)sides);
+  kern<<<grid, kEncThreads, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
 template <int KB, int VB>
 int launch_kb_vb(const EncodeParams& p, cudaStream_t stream) {
   const long long n_blocks = (long long)p.batch * p.kv_heads * p.seq_new * (p.head_dim / kBlock);
-  const long long threads = n_blocks * 2;
-  const long long grid_x = (threads + kEncThreads - 1) / kEncThreads;
-  if (grid_x > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)grid_x, 2);
+  if (n_blocks >= (1LL << 31)) return TQ_ERR_UNSUPPORTED;  // 32-bit index math in the kernel
   const bool outl = p.vo_k > 0 && p.in[1] != nullptr;
+  const int sides = (p.in[0] ? 1 : 0) + (p.in[1] ? 1 : 0);
   if (p.f16) {
-    if (outl) encode_kernel<KB, VB, true, true><<<grid, kEncThreads, 0, stream>>>(p);
-    else encode_kernel<KB, VB, true, false><<<grid, kEncThreads, 0, stream>>>(p);
-  } else {
-    if (outl) encode_kernel<KB, VB, false, true><<<grid, kEncThreads, 0, stream>>>(p);
-    else encode_kernel<KB, VB, false, false><<<grid, kEncThreads, 0, stream>>>(p);
+    if (outl) return launch_typed(encode_kernel<KB, VB, true, true>, stage_bytes<true>(), p, n_blocks, sides, stream);
+    return launch_typed(encode_kernel<KB, VB, true, false>, stage_bytes<true>(), p, n_blocks, sides, stream);
   }
-  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  if (outl) return launch_typed(encode_kernel<KB, VB, false, true>, stage_bytes<false>(), p, n_blocks, sides, stream);
+  return launch_typed(encode_kernel<KB, VB, false, false>, stage_bytes<false>(), p, n_blocks, sides, stream);
 }
 
 template <int KB>

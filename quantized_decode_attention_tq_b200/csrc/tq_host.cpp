@@ -352,6 +352,8 @@ int tq_encode_kv_v3(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_co
   p.head_dim = desc->head_dim;
   p.seq_cap = desc->seq_cap;
   p.seq_new = seq_new;
+  p.div_seq_new = tq::FastDiv::make((uint32_t)seq_new);
+  p.div_kv_heads = tq::FastDiv::make((uint32_t)desc->kv_heads);
   if (vo && vo->k > 0) {
     p.vo_k = vo->k;
     p.vo_kp = outlier_row(vo->k);

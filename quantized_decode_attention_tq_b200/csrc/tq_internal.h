@@ -18,6 +18,30 @@ constexpr int kMaxBatch = 2048;    // decode batch limit (the tile prefix lives 
 constexpr int kMaxHeadDim = 512;   // encoder: up to 4 blocks per vector
 constexpr int kMaxDecodeHeadDim = 256;  // decode kernels are built for 1 or 2 blocks
 
+// Division of 32-bit unsigned n by a fixed d >= 1 without a divide: with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1, t = mulhi(m, n)
+// gives n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0) for every n
+// below 2^32 (Granlund and Montgomery, PLDI 1994, figure 4.1).
+struct FastDiv {
+  uint32_t d, m, s1, s2;
+  static FastDiv make(uint32_t div) {
+    FastDiv f{};
+    f.d = div;
+    int l = 0;
+    while ((1ull << l) < div) ++l;
+    f.m = (uint32_t)((((1ull << l) - div) << 32) / div + 1);
+    f.s1 = l > 0 ? 1u : 0u;
+    f.s2 = l > 1 ? (uint32_t)(l - 1) : 0u;
+    return f;
+  }
+#ifdef __CUDACC__
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    const uint32_t t = __umulhi(m, n);
+    return (t + ((n - t) >> s1)) >> s2;
+  }
+#endif
+};
+
 // Encoder launch parameters (one launch writes K and V).
 struct EncodeParams {
   const void* in[2];          // K, V inputs [B, Hkv, seq_new, D] (either may be null)
@@ -30,6 +54,7 @@ struct EncodeParams {
   uint32_t sign_mask[4];      // bit i set <=> s_i = -1
   int f16;                    // input dtype: 1 = fp16, 0 = fp32
   int batch, kv_heads, head_dim, seq_cap, seq_new;
+  FastDiv div_seq_new, div_kv_heads;  // index splits of the flattened rows (below 2^31)
   // V v3 (vo_k > 0): channels [kv_heads, vo_k] of V are zeroed before the
   // encoding and their values written to vo_values [.., seq_cap, vo_kp]
   const int32_t* vo_channels;
