@@ -12,7 +12,7 @@
 //  * Work = (unit, 16-token tile), unit = (batch, kv-head, group of <= 8
 //    query heads).  All tiles of all units are laid end to end and cut into
 //    one range per persistent CTA, one 16-warp CTA per SM.  The cut weighs each
-//    tile 1 and each unit start kSwitchTiles more (see Split).  A CTA writes
+//    tile 1 and each unit boundary more (see Split).  A CTA writes
 //    one partial (m, l, acc) per unit it touches; the CTA that completes a unit
 //    (atomic tile count) merges the partials in a fixed order, so results do
 //    not depend on scheduling.
@@ -38,8 +38,16 @@
 //    pair of adjacent dims straight from the table.  With more heads (GQ = 8)
 //    V is re-paired by token.  V stays in the rotated domain until the end.
 //  * Sparse-V is exact and two-pass: pass 1 stores log2-domain scores and
-//    per-partial (m, l); pass 2 forms the log-sum-exp, zeroes the normalised
-//    weights below the threshold and accumulates V with the rest.
+//    per-partial (m, l); pass 2 forms each head's maximum M and log-sum-exp,
+//    drops the positions whose normalised weight 2^(s - LSE) is below the
+//    threshold and accumulates V with weights 2^(s - M - 7), as the fused
+//    pass does, dividing by the head's sum at the end.
+//  * V v3 (VO): each tile also carries its 16 tokens' outlier-channel values
+//    (fp16); one more MMA per tile sums them with the plain weights, and the
+//    emit overwrites those channels of the output.
+//  * V v2 (V2): the V codes are trellis pair fields; a pair's two levels are
+//    indexed by the stream bits that end with its field (the two branch bits
+//    before it included), so V fragments come from pair tables as in v1.
 //  * The tail has no block-wide merge stage: warp h merges the 16 warps'
 //    partials of head h and either emits the head (inverse rotation in
 //    registers) or publishes the CTA's partial; the completing CTA's warp h
@@ -60,6 +68,9 @@ namespace {  // every including translation unit keeps its own copy
 #ifndef TQ_SWITCH_TILES
 #define TQ_SWITCH_TILES 96  // cost of starting another unit inside a CTA, in tiles
 #endif
+#ifndef TQ_APPEND_TILES
+#define TQ_APPEND_TILES 32  // extra cost of a unit end whose CTA appends the new token, in tiles
+#endif
 #ifndef TQ_KCHAINS
 #define TQ_KCHAINS 2  // independent accumulator chains of the score MMAs
 #endif
@@ -72,6 +83,8 @@ constexpr uint32_t kMaxDyn = 227 * 1024;
 constexpr float kTau = 6.0f;            // lazy-rescale threshold (log2 units)
 constexpr float kPShift = 7.0f;         // weights carry 2^-7 = 1/128
 constexpr long long kSwitchTiles = TQ_SWITCH_TILES;
+constexpr long long kAppendTiles = TQ_APPEND_TILES;
+constexpr long long kMinCtaTiles = 32;  // a CTA per this many tiles at most (two per warp)
 
 enum Mode { kFused = 0, kScores = 1, kSparseV = 2 };
 
@@ -382,11 +395,13 @@ __device__ __noinline__ void append_block(const DecodeParams& p, int side, int b
 }
 
 // How the flattened (unit, tile) space [0, T) is split over the persistent
-// CTAs.  Every unit's tiles cost 1 each and starting a unit costs kSwitchTiles
-// more (its query preparation, the drained copy ring, the partial's merge
-// and publication), so a CTA whose range spans two units gets fewer tiles:
-// CTA c takes the tiles whose cost falls in [c, c+1) * Ctot / P.  The cost
-// before batch entry b is UB * (prefix[b] + kSwitchTiles * b).  A cost that
+// CTAs.  Every unit's tiles cost 1 each and each unit boundary costs sw more
+// (kSwitchTiles: the query preparation, the drained copy ring, the partial's
+// merge and publication; plus kAppendTiles in a decode step, whose CTA that
+// holds a unit's last tile first appends the new token), so a CTA whose range
+// spans a boundary gets fewer tiles: CTA c takes the tiles whose cost falls in
+// [c, c+1) * Ctot / P.  The cost before batch entry b is
+// UB * (prefix[b] + sw * b).  A cost that
 // falls between two units maps to the start of the second, so a cut there
 // adds no segment.  Results do not depend on the split (each part is computed
 // and merged in a fixed order); it only moves where the CTAs end.
@@ -414,12 +429,12 @@ __device__ __forceinline__ long long qdiv_small(long long a, long long b) {
 struct Split {
   const int* prefix;  // [B+1] tiles per batch entry, exclusive prefix (shared memory)
   int B, UB;
-  long long P, T, Ctot;
+  long long P, T, Ctot, sw;
   double invP, invCtot, invUB;
-  __device__ Split(const int* pre, int batch, int ub, long long parts)
-      : prefix(pre), B(batch), UB(ub), P(parts) {
+  __device__ Split(const int* pre, int batch, int ub, long long parts, long long switch_cost)
+      : prefix(pre), B(batch), UB(ub), P(parts), sw(switch_cost) {
     T = (long long)pre[batch] * ub;
-    Ctot = (long long)ub * ((long long)pre[batch] + kSwitchTiles * batch);
+    Ctot = (long long)ub * ((long long)pre[batch] + sw * batch);
     invP = 1.0 / (double)P;
     invCtot = Ctot > 0 ? 1.0 / (double)Ctot : 0.0;
     invUB = 1.0 / (double)ub;
@@ -431,11 +446,11 @@ struct Split {
     int bl = 0, bh = B;  // largest b with cost(b) <= y
     while (bh - bl > 1) {
       const int mid = (bl + bh) >> 1;
-      if ((long long)UB * (prefix[mid] + kSwitchTiles * mid) <= y) bl = mid; else bh = mid;
+      if ((long long)UB * (prefix[mid] + sw * mid) <= y) bl = mid; else bh = mid;
     }
     const long long nt = prefix[bl + 1] - prefix[bl];
-    const long long rem = y - (long long)UB * (prefix[bl] + kSwitchTiles * bl);
-    const long long r = qdiv_small(rem, nt + kSwitchTiles), t = rem - r * (nt + kSwitchTiles);
+    const long long rem = y - (long long)UB * (prefix[bl] + sw * bl);
+    const long long r = qdiv_small(rem, nt + sw), t = rem - r * (nt + sw);
     return (long long)UB * prefix[bl] + r * nt + min(t, nt);
   }
   // The part whose range holds tile x (0 <= x < T): the last c whose cost
@@ -449,7 +464,7 @@ struct Split {
     const long long nt = prefix[bl + 1] - prefix[bl];
     const long long off = x - (long long)UB * prefix[bl];
     const long long r = qdiv_small(off, nt), t = off - r * nt;
-    const long long F = (long long)UB * (prefix[bl] + kSwitchTiles * bl) + r * (nt + kSwitchTiles) + t;
+    const long long F = (long long)UB * (prefix[bl] + sw * bl) + r * (nt + sw) + t;
     const long long c = qdiv((F + 1) * P - 1, Ctot, invCtot);
     return c < P - 1 ? c : P - 1;
   }
@@ -814,7 +829,9 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     if (tid == kThreads - 1) prefix[B] = run;
     __syncthreads();  // also publishes the tables and the barrier initialisation
   }
-  const Split sp(prefix, p.batch, UB, gridDim.x);  // this launch's split
+  // the cost of a unit boundary: a decode step (new rows given) appends there
+  const long long sw = kSwitchTiles + (p.kv_new[0] != nullptr ? kAppendTiles : 0);
+  const Split sp(prefix, p.batch, UB, gridDim.x, sw);  // this launch's split
   const long long T = sp.T;
 
   const long long lo = T > 0 ? sp.start(blockIdx.x) : 0, hi = T > 0 ? sp.start(blockIdx.x + 1) : 0;
@@ -1088,7 +1105,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       tables_ready = true;
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote; warp hd takes head hd
-      const Split sp1(prefix, p.batch, UB, p1_ctas);
+      const Split sp1(prefix, p.batch, UB, p1_ctas, sw);  // pass 1 had the same parameters
       if (cw < Gu) {
         const float2 ML = unit_ml_warp(p.slot_ml, sp1.part_of(Su), sp1.part_of(Su + nt - 1), sp1, unit, cw, lane);
         if (lane == 0) {
@@ -1496,7 +1513,11 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         // this CTA saw the entire unit: no partial needed
         emit_row(v, ov, (MODE == kFused ? L : u_l[hd]) * 128.0f, b, h0 + hd);
       } else {
-        if (lane == 0)
+        // (m, l) of the partial: the fused merge weighs by it and pass 2 of
+        // sparse-V reads pass 1's.  Pass 2 itself writes none: its CTAs read
+        // pass 1's (m, l) at each segment start, and a write to the same slot
+        // could land before another CTA's read.
+        if (lane == 0 && MODE != kSparseV)
           *reinterpret_cast<float2*>(p.slot_ml + (slot * kMaxGroup + hd) * 2) = make_float2(M, L);
         if constexpr (HASV) {
 #pragma unroll
@@ -1742,7 +1763,14 @@ int run(DecodeParams& p, cudaStream_t stream, int p1_ctas, int* ctas_out) {
     cached_smem[dev] = kMaxDyn;
     cached_sms[dev] = sms;
   }
-  const int ctas = min(kMaxCtas, cached_sms[dev]);
+  // one CTA per SM, but no more than one per kMinCtaTiles tiles of the
+  // largest launch these sizes allow (a short cache is done by fewer CTAs,
+  // with fewer partials to merge)
+  const long long n_hg = (p.q_heads / p.kv_heads * p.n_q + kMaxGroup - 1) / kMaxGroup;
+  const long long tiles_max = (long long)p.batch * p.kv_heads * n_hg * ((p.seq_cap + kTile - 1) / kTile);
+  int ctas = min(kMaxCtas, cached_sms[dev]);
+  if ((tiles_max + kMinCtaTiles - 1) / kMinCtaTiles < ctas)
+    ctas = (int)max(1LL, (tiles_max + kMinCtaTiles - 1) / kMinCtaTiles);
   kern<<<ctas, kThreads, smem, stream>>>(p, p1_ctas);
   if (cudaGetLastError() != cudaSuccess) return TQ_ERR_CUDA;
   if (ctas_out) *ctas_out = ctas;

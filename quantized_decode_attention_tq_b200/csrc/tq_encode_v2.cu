@@ -106,7 +106,14 @@ encode_v2_kernel(const __grid_constant__ EncodeParams p) {
   constexpr int NW = 4 * BITS;          // 32-bit words of a block's codes
   __shared__ float su[kV2Warps][32][kURow];
   __shared__ uint32_t sdec[kV2Warps][32][kDecRow];
+  __shared__ __align__(16) float smid[4][4];  // decision points of each subset, for the traceback
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x < 16) {
+    const int k = threadIdx.x >> 2, m = threadIdx.x & 3;
+    smid[k][m] = m + 1 < (1 << (BITS - 1)) ? 0.5f * (p.tcq_levels[4 * m + k] + p.tcq_levels[4 * (m + 1) + k])
+                                           : INFINITY;
+  }
+  __syncthreads();
   const int nb = p.head_dim / kBlock;
   const long long n_items = (long long)p.batch * p.kv_heads * p.seq_new * nb;
   const long long first = ((long long)blockIdx.x * kV2Warps + warp) * 32;
@@ -115,31 +122,38 @@ encode_v2_kernel(const __grid_constant__ EncodeParams p) {
   for (int e = 0; e < 4; ++e) sgn |= ((p.sign_mask[e] >> lane) & 1u) << e;
   const void* in = p.in[1];
 
-  // ---- rotation and norm, one block at a time by the whole warp ----------
+  // ---- rotation and norm by the whole warp, eight blocks' loads in flight
+  // at a time (the warp's 32 blocks are one contiguous input range) ---------
   float my_norm = 0.0f;
-  for (int i = 0; i < 32; ++i) {
-    const long long item = first + i;
-    if (item >= n_items) break;  // warp-uniform
-    const long long row = item / nb;
-    const int blk = (int)(item % nb);
-    const size_t off = (size_t)row * p.head_dim + (size_t)blk * kBlock + lane;
-    float v[4];
+  for (int g0 = 0; g0 < 32; g0 += 8) {
+    if (first + g0 >= n_items) break;  // warp-uniform
+    float v8[8][4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      v[e] = F16 ? __half2float(static_cast<const __half*>(in)[off + 32 * e])
-                 : static_cast<const float*>(in)[off + 32 * e];
+    for (int i = 0; i < 8; ++i) {
+      const long long item = first + g0 + i;
+      const size_t off = (size_t)item * kBlock + lane;  // item * 128 = row * D + blk * 128
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if ((sgn >> e) & 1u) v[e] = -v[e];
-    float ss = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+      for (int e = 0; e < 4; ++e)
+        v8[i][e] = item >= n_items ? 0.0f
+                   : F16 ? __half2float(static_cast<const __half*>(in)[off + 32 * e])
+                         : static_cast<const float*>(in)[off + 32 * e];
+    }
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-    const float n = sqrtf(ss);
-    wht_block(v, lane);
-    const float inv = n > 0.0f ? 1.0f / n : 0.0f;  // u = 0 for a zero block
+    for (int i = 0; i < 8; ++i) {
+      float (&v)[4] = v8[i];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) su[warp][i][lane + 32 * e] = v[e] * inv;
-    if (lane == i) my_norm = n;
+      for (int e = 0; e < 4; ++e)
+        if ((sgn >> e) & 1u) v[e] = -v[e];
+      float ss = v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3];
+#pragma unroll
+      for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      const float n = sqrtf(ss);
+      wht_block(v, lane);
+      const float inv = n > 0.0f ? 1.0f / n : 0.0f;  // u = 0 for a zero block
+#pragma unroll
+      for (int e = 0; e < 4; ++e) su[warp][g0 + i][lane + 32 * e] = v[e] * inv;
+      if (lane == g0 + i) my_norm = n;
+    }
   }
   __syncwarp();
 
@@ -205,10 +219,11 @@ encode_v2_kernel(const __grid_constant__ EncodeParams p) {
       const int pred = d ? ((s >> 1) | 2) : (s >> 1);
       const int beta = s & 1;
       const int sub = (pred & 1) + 2 * (beta ^ (pred >> 1));
-      float l;
-      const int j0 = tc.nearest(u[i], 0, l), j1 = tc.nearest(u[i], 1, l);
-      const int j2 = tc.nearest(u[i], 2, l), j3 = tc.nearest(u[i], 3, l);
-      jj[q] = (uint32_t)(sub == 0 ? j0 : sub == 1 ? j1 : sub == 2 ? j2 : j3);
+      // the level index in the subset: #{decision points below u} (the same
+      // points the forward search compared with; unused slots are +inf)
+      const float4 md = *reinterpret_cast<const float4*>(smid[sub]);
+      const float x = u[i];
+      jj[q] = (x > md.x ? 1u : 0u) + (x > md.y ? 1u : 0u) + (x > md.z ? 1u : 0u);
       bb[q] = (uint32_t)beta;
       s = pred;
     }

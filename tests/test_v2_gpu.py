@@ -208,3 +208,45 @@ def test_v2_beats_the_plain_format_at_the_same_rate(vb):
     r2 = O.dequantize_v2(vc2, vn2, vb, O.tcq_levels_f32(vb), sg)
     r1 = O.dequantize(vc1, vn1, vb, O.codebook_f32(vb)[0], sg)
     assert snr_db(r2, x) > snr_db(r1, x) + 0.5
+
+
+def test_decode_v2_edge_lengths():
+    # an empty sequence (zero row), a single position (the trellis's first
+    # step), and a full cache
+    w = inputs.make("gqa", batch=3, seq=96)
+    lens = [0, 1, 96]
+    cache, kcb, vtq = _encode_v2(w)
+    o_gpu = _decode_v2(cache, kcb, vtq, w.q, lens, w.scale)
+    assert np.all(o_gpu[0] == 0.0)
+    check_decode(o_gpu[1:], _oracle_v2(w, cache, lens, 0.0)[1:])
+
+
+@pytest.mark.parametrize("name,units", [("gqa", [(0, 0), (6, 2)]), ("ragged", [(0, 1), (3, 3)])])
+def test_decode_v2_full_sampled(name, units):
+    """Full workloads in the benchmark's launch shape (GQA K3/V3; ragged K3/V2
+    D256 with sparse-V); sampled (batch, kv-head) units against the oracle."""
+    w = inputs.make(name)
+    cache, kcb, vtq = _encode_v2(w)
+    o_gpu = _decode_v2(cache, kcb, vtq, w.q, w.seq_lens, w.scale, w.sparse_thr)
+    kc, kn, vc, vn = host(cache)
+    g = w.q_heads // w.kv_heads
+    for b, h in units:
+        sl = slice(h, h + 1)
+        qs = w.q[b:b + 1, h * g:(h + 1) * g].astype(np.float64)
+        o_ref = O.decode_v2_rotated(qs, kc[b:b + 1, sl], kn[b:b + 1, sl], vc[b:b + 1, sl], vn[b:b + 1, sl],
+                                    w.seq_lens[b:b + 1], w.scale, w.k_bits, w.v_bits,
+                                    O.codebook_f32(w.k_bits)[0], O.tcq_levels_f32(w.v_bits),
+                                    O.sign_vector(w.sign_seed), w.sparse_thr)
+        bound = None
+        if w.sparse_thr > 0:
+            kt = O.dequantize(kc[b:b + 1, sl], kn[b:b + 1, sl], w.k_bits, O.codebook_f32(w.k_bits)[0],
+                              O.sign_vector(w.sign_seed))
+            vt = O.dequantize_v2(vc[b:b + 1, sl], vn[b:b + 1, sl], w.v_bits, O.tcq_levels_f32(w.v_bits),
+                                 O.sign_vector(w.sign_seed))
+            wts = O.attention_weights(qs, kt, w.seq_lens[b:b + 1], w.scale)
+            bound = np.zeros(qs.shape)
+            n = int(w.seq_lens[b])
+            for (bb, hh), wt in wts.items():
+                amb = np.abs(np.log(np.maximum(wt, 1e-300) / w.sparse_thr)) < SPARSE_BAND
+                bound[bb, hh] = wt[amb] @ np.abs(vt[bb, 0, :n][amb])
+        check_decode(o_gpu[b:b + 1, h * g:(h + 1) * g], o_ref, bound)

@@ -280,3 +280,35 @@ def test_v3_channel_out_of_range_sets_status():
     vo2 = tq.VOutliers(2, to_dev(valid.astype(np.int32)), vo.values[..., :8].contiguous())
     o_ref = _oracle_v3(w, cache, vo2, [64], 0.0)
     _check_v3_decode(o_gpu, o_ref, valid, w.q_heads // w.kv_heads)
+
+
+def test_decode_v3_edge_lengths():
+    # an empty sequence (zero row), a single position, and a full cache
+    w = inputs.make("gqa", batch=3, seq=96, dist="outlier_v")
+    lens = [0, 1, 96]
+    cache, kcb, vcb, vo = _encode_v3(w, 5)
+    o_gpu = _decode_v3(cache, kcb, vcb, vo, w.q, lens, w.scale)
+    assert np.all(o_gpu[0] == 0.0)
+    o_ref = _oracle_v3(w, cache, vo, lens, 0.0)
+    _check_v3_decode(o_gpu[1:], o_ref[1:], vo.channels.cpu().numpy(), w.q_heads // w.kv_heads)
+
+
+def test_decode_v3_full_gqa_sampled():
+    """The full GQA workload (B8, S32768) with outlier-channel V, k = 8, in the
+    benchmark's launch shape; sampled (batch, kv-head) units against the oracle."""
+    w = inputs.make("gqa", dist="outlier_v")
+    cache, kcb, vcb, vo = _encode_v3(w, 8)
+    o_gpu = _decode_v3(cache, kcb, vcb, vo, w.q, w.seq_lens, w.scale)
+    kc, kn, vc, vn = host(cache)
+    vals = vo.values.cpu().numpy().view(np.float16)[..., : vo.k]
+    ch = vo.channels.cpu().numpy()
+    g = w.q_heads // w.kv_heads
+    kcent, _ = O.codebook_f32(w.k_bits)
+    vcent, _ = O.codebook_f32(w.v_bits)
+    for b, h in [(0, 0), (5, 3), (7, 7)]:
+        sl = slice(h, h + 1)
+        qs = w.q[b:b + 1, h * g:(h + 1) * g].astype(np.float64)
+        o_ref = O.decode_v3_rotated(qs, kc[b:b + 1, sl], kn[b:b + 1, sl], vc[b:b + 1, sl], vn[b:b + 1, sl],
+                                    vals[b:b + 1, sl], ch[sl], w.seq_lens[b:b + 1], w.scale, w.k_bits, w.v_bits,
+                                    kcent, vcent, O.sign_vector(w.sign_seed))
+        _check_v3_decode(o_gpu[b:b + 1, h * g:(h + 1) * g], o_ref, ch[sl], g)
