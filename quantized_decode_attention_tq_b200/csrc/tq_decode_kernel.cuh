@@ -69,7 +69,7 @@ namespace {  // every including translation unit keeps its own copy
 #define TQ_SWITCH_TILES 96  // cost of starting another unit inside a CTA, in tiles
 #endif
 #ifndef TQ_APPEND_TILES
-#define TQ_APPEND_TILES 32  // extra cost of a unit end whose CTA appends the new token, in tiles
+#define TQ_APPEND_TILES 64  // extra cost of a unit end whose CTA appends the new token, in tiles
 #endif
 #ifndef TQ_KCHAINS
 #define TQ_KCHAINS 2  // independent accumulator chains of the score MMAs
