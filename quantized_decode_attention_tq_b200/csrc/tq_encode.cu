@@ -338,12 +338,12 @@ __device__ __forceinline__ void encode_block(const EncodeParams& p, const uint32
 
 template <int BITS, bool F16, int SIDE, bool OUTL>
 __device__ __forceinline__ void encode_side(const EncodeParams& p, const uint32_t* ws, uint32_t st0,
-                                            uint32_t n_blocks) {
+                                            uint32_t n_blocks, uint32_t cta, uint32_t ctas) {
   const int lane = threadIdx.x & 31;
-  // lane pairs walk the blocks with a grid stride; the warp stays together
-  // (its pairs are consecutive) so the loop is warp-uniform
-  const uint32_t pairs = (gridDim.x * blockDim.x) >> 1;
-  const uint32_t warp0 = (blockIdx.x * blockDim.x + (threadIdx.x & ~31u)) >> 1;
+  // lane pairs walk the blocks with a stride of this side's lane pairs; the
+  // warp stays together (its pairs are consecutive) so the loop is warp-uniform
+  const uint32_t pairs = (ctas * blockDim.x) >> 1;
+  const uint32_t warp0 = (cta * blockDim.x + (threadIdx.x & ~31u)) >> 1;
   const uint32_t mine = lane >> 1;
   if (warp0 >= n_blocks) return;
   stage_block<F16>(p, p.in[SIDE], warp0 + mine, n_blocks, st0, lane);
@@ -377,16 +377,21 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_consta
   }
   const uint32_t st0 = (uint32_t)__cvta_generic_to_shared(stage) + (uint32_t)warp * 2u * stage_bytes<F16>();
   const uint32_t n_blocks = (uint32_t)p.batch * p.kv_heads * p.seq_new * (p.head_dim / kBlock);
-  // grid.y: both sides (y = side) or the one side present
-  const int side = gridDim.y == 2 ? (int)blockIdx.y : (p.in[0] ? 0 : 1);
-  if (side == 0) encode_side<KB, F16, 0, false>(p, ws, st0, n_blocks);
-  else encode_side<VB, F16, 1, OUTL>(p, ws, st0, n_blocks);
+  // the first k_ctas CTAs encode K, the rest V (k_ctas = 0: V only; all: K only)
+  const uint32_t kc = p.k_ctas;
+  if (blockIdx.x < kc) encode_side<KB, F16, 0, false>(p, ws, st0, n_blocks, blockIdx.x, kc);
+  else encode_side<VB, F16, 1, OUTL>(p, ws, st0, n_blocks, blockIdx.x - kc, gridDim.x - kc);
 }
 
-// Persistent launch: as many CTAs as are resident at once (split between the
-// sides), at most one lane pair per block.
+// Instructions per element by code width, for splitting the CTAs between K
+// and V in proportion to their work: the transform, loads and packing (about
+// 12) plus the quantiser's compares and bit toggles.
+inline int side_cost(int bits) { return 12 + (bits == 2 ? 4 : bits == 3 ? 7 : 11); }
+
+// Persistent launch: as many CTAs as are resident at once, split between the
+// sides in proportion to their work, at most one lane pair per block.
 template <typename K>
-int launch_typed(K kern, uint32_t stage, const EncodeParams& p, long long n_blocks, int sides, cudaStream_t stream) {
+int launch_typed(K kern, uint32_t stage, EncodeParams p, long long n_blocks, cudaStream_t stream) {
   const size_t smem = (size_t)(kEncThreads / 32) * 2 * stage;
   int dev = 0, sms = 0, occ = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
@@ -395,10 +400,22 @@ int launch_typed(K kern, uint32_t stage, const EncodeParams& p, long long n_bloc
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TQ_ERR_CUDA;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kEncThreads, smem) != cudaSuccess) return TQ_ERR_CUDA;
   if (occ < 1) return TQ_ERR_UNSUPPORTED;
-  const long long per_side = std::max(1LL, (long long)occ * sms / sides);
-  const long long needed = (n_blocks * 2 + kEncThreads - 1) / kEncThreads;
-  dim3 grid((unsigned)std::min(per_side, needed), (unsigned)sides);
-  kern<<<grid, kEncThreads, smem, stream>>>(p);
+  const long long needed = (n_blocks * 2 + kEncThreads - 1) / kEncThreads;  // CTAs one side can use
+  const long long resident = (long long)occ * sms;
+  long long kc = 0, vc = 0;
+  if (p.in[0] && p.in[1]) {
+    const int ck = side_cost(p.bits[0]), cv = side_cost(p.bits[1]);
+    kc = std::max(1LL, std::min(resident - 1, (resident * ck + (ck + cv) / 2) / (ck + cv)));
+    vc = std::max(1LL, resident - kc);
+  } else if (p.in[0]) {
+    kc = resident;
+  } else {
+    vc = resident;
+  }
+  kc = std::min(kc, needed);
+  vc = std::min(vc, needed);
+  p.k_ctas = (uint32_t)kc;
+  kern<<<(unsigned)(kc + vc), kEncThreads, smem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
@@ -407,13 +424,12 @@ int launch_kb_vb(const EncodeParams& p, cudaStream_t stream) {
   const long long n_blocks = (long long)p.batch * p.kv_heads * p.seq_new * (p.head_dim / kBlock);
   if (n_blocks >= (1LL << 31)) return TQ_ERR_UNSUPPORTED;  // 32-bit index math in the kernel
   const bool outl = p.vo_k > 0 && p.in[1] != nullptr;
-  const int sides = (p.in[0] ? 1 : 0) + (p.in[1] ? 1 : 0);
   if (p.f16) {
-    if (outl) return launch_typed(encode_kernel<KB, VB, true, true>, stage_bytes<true>(), p, n_blocks, sides, stream);
-    return launch_typed(encode_kernel<KB, VB, true, false>, stage_bytes<true>(), p, n_blocks, sides, stream);
+    if (outl) return launch_typed(encode_kernel<KB, VB, true, true>, stage_bytes<true>(), p, n_blocks, stream);
+    return launch_typed(encode_kernel<KB, VB, true, false>, stage_bytes<true>(), p, n_blocks, stream);
   }
-  if (outl) return launch_typed(encode_kernel<KB, VB, false, true>, stage_bytes<false>(), p, n_blocks, sides, stream);
-  return launch_typed(encode_kernel<KB, VB, false, false>, stage_bytes<false>(), p, n_blocks, sides, stream);
+  if (outl) return launch_typed(encode_kernel<KB, VB, false, true>, stage_bytes<false>(), p, n_blocks, stream);
+  return launch_typed(encode_kernel<KB, VB, false, false>, stage_bytes<false>(), p, n_blocks, stream);
 }
 
 template <int KB>

@@ -55,6 +55,7 @@ struct EncodeParams {
   int f16;                    // input dtype: 1 = fp16, 0 = fp32
   int batch, kv_heads, head_dim, seq_cap, seq_new;
   FastDiv div_seq_new, div_kv_heads;  // index splits of the flattened rows (below 2^31)
+  uint32_t k_ctas;                    // CTAs of the launch that encode K (set by launch_encode)
   // V v3 (vo_k > 0): channels [kv_heads, vo_k] of V are zeroed before the
   // encoding and their values written to vo_values [.., seq_cap, vo_kp]
   const int32_t* vo_channels;
