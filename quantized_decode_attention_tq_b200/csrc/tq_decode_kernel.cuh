@@ -794,16 +794,24 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     if constexpr (HASV && !V2)
       fill_table(VB, p.vcent, VB == 3 ? sm.lut_v : sm.lut_v & ~255u, VB == 3 ? 0u : (sm.lut_v & 128u), t_first, t_count);
   };
-  bool tables_ready = false;  // filled during the first segment's query preparation
 
   // ---- lengths: clamp, tiles per batch entry, exclusive prefix ------------
+  // (the code tables are filled while this thread's length loads are in
+  // flight; the barrier below publishes them)
   {
     const int B = p.batch;
-    const int per = (B + kThreads - 1) / kThreads;
+    const int per = (B + kThreads - 1) / kThreads;  // at most kMaxBatch / kThreads = 4
     int local = 0;
     const int b_lo = tid * per;
-    for (int b = b_lo; b < min(B, b_lo + per); ++b) {
-      int len = __ldg(p.seq_lens + b);
+    int lens_r[kMaxBatch / kThreads];
+#pragma unroll
+    for (int i = 0; i < kMaxBatch / kThreads; ++i)
+      lens_r[i] = (i < per && b_lo + i < B) ? __ldg(p.seq_lens + b_lo + i) : 0;
+    fill_tables(0, kThreads);
+#pragma unroll
+    for (int i = 0; i < kMaxBatch / kThreads; ++i) {
+      if (i >= per || b_lo + i >= B) break;
+      int len = lens_r[i];
       if (len < 0 || len > p.seq_cap) {
         if (blockIdx.x == 0 && p.status) atomicOr(p.status, TQ_DEV_LEN_RANGE);
         len = min(max(len, 0), p.seq_cap);
@@ -914,8 +922,6 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   auto prep_q = [&](int b, int h0, int Gu, uint32_t (&qf)[NB][8][2], float (&qmul)[2]) {
     constexpr int kQRows = kDup ? 4 : kMaxGroup;
     float* qs = res;  // [kQRows] rows of scaled qhat (QScratch layout)
-    // the first segment's idle warps fill the code tables meanwhile
-    if (!tables_ready) fill_tables(32 * kQRows, kThreads - 32 * kQRows);
     for (int j = cw; j < kQRows; j += kCWarps) {
       float v[NB][4];
 #pragma unroll
@@ -966,7 +972,6 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
         qf[blk][j][1] = pack_half2(q4.z, q4.w);
       }
     }
-    tables_ready = true;
     qmul[0] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g) & 3 : 2 * g]);
     qmul[1] = p.score_mult * ldexpf(1.0f, qexp[kDup ? (2 * g + 1) & 3 : 2 * g + 1]);
     consumer_sync();  // res and qexp are reused after this
@@ -1101,8 +1106,6 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     float lse2[2] = {0.0f, 0.0f}, moff2[2] = {0.0f, 0.0f};
     if constexpr (HASK) prep_q(b, h0, Gu, qf, qmul);
     if constexpr (MODE == kSparseV) {
-      if (!tables_ready) fill_tables(0, kThreads);
-      tables_ready = true;
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote; warp hd takes head hd
       const Split sp1(prefix, p.batch, UB, p1_ctas, sw);  // pass 1 had the same parameters
@@ -1544,20 +1547,12 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             const float* ml_base = p.slot_ml + ((long long)unit * kMaxGroup + hd) * 2;
             const float* acc_base = p.slot_acc + ((long long)unit * kMaxGroup + hd) * PD + 4 * lane;
             const long long ml_stride = kMaxGroup * 2, part_stride = (long long)kMaxGroup * PD;
-            // pass 1: the maximum over the partials (lane j holds part c0 + j)
-            float Mx = -INFINITY;
-            if constexpr (MODE == kFused) {
-              for (long long c0 = c_first; c0 <= c_last; c0 += 32) {
-                const uint32_t emp = empty_bits(sp, c0, c_last, lane);
-                const long long c = c0 + lane;
-                if (c <= c_last && !((emp >> lane) & 1u)) Mx = fmaxf(Mx, __ldcg(ml_base + c * ml_stride));
-              }
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, o));
-            }
-            // pass 2: weights 2^(m_c - M), then every partial's acc in part
-            // order with all loads of a 32-part chunk in flight
-            float Lx = 0.0f;
+            // One pass over the partials in chunks of 32 (lane j holds part
+            // c0 + j): the chunk's (m, l) give its maximum; a chunk whose
+            // maximum exceeds the running one rescales what came before (no
+            // rescale with a single chunk, the common case); then every
+            // partial's acc is added in part order with the loads in flight.
+            float Mx = -INFINITY, Lx = 0.0f;
             float u[NB][4];
 #pragma unroll
             for (int blk = 0; blk < NB; ++blk)
@@ -1567,18 +1562,27 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
             for (long long c0 = c_first; c0 <= c_last; c0 += 32) {
               const uint32_t emp = empty_bits(sp, c0, c_last, lane);
               const long long c = c0 + lane;
-              float wgt = 0.0f;
-              float lw = 0.0f;
-              if (c <= c_last && !((emp >> lane) & 1u)) {
-                if constexpr (MODE == kFused) {
-                  const float2 ml = __ldcg(reinterpret_cast<const float2*>(ml_base + c * ml_stride));
-                  wgt = (ml.x == -INFINITY) ? 0.0f : ex2(ml.x - Mx);
-                  lw = wgt != 0.0f ? ml.y * wgt : 0.0f;
-                } else {
-                  wgt = 1.0f;
+              const bool live = c <= c_last && !((emp >> lane) & 1u);
+              float wgt = live ? 1.0f : 0.0f;
+              if constexpr (MODE == kFused) {
+                const float2 ml = live ? __ldcg(reinterpret_cast<const float2*>(ml_base + c * ml_stride))
+                                       : make_float2(-INFINITY, 0.0f);
+                float cm = ml.x;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+                if (cm > Mx) {  // warp-uniform
+                  const float sc = (Mx == -INFINITY) ? 0.0f : ex2(Mx - cm);
+                  Lx *= sc;
+#pragma unroll
+                  for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) u[blk][k] *= sc;
+#pragma unroll
+                  for (int k = 0; k < 4; ++k) uo[k] *= sc;
+                  Mx = cm;
                 }
-              }
-              if constexpr (MODE == kFused) {  // L: fixed-order reduction over the chunk
+                wgt = (ml.x == -INFINITY) ? 0.0f : ex2(ml.x - Mx);
+                float lw = wgt != 0.0f ? ml.y * wgt : 0.0f;  // L: fixed-order reduction over the chunk
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
                 Lx += lw;

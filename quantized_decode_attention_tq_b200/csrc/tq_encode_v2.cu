@@ -19,14 +19,17 @@
 //     j_2k, j_2k+1 (b - 1 bits each), then beta_2k, beta_2k+1.
 // The block norm and rotation are those of the v1 encoder.
 //
-// Mapping: a warp takes 32 blocks.  Block by block, the warp loads it (lane l:
-// elements l, l + 32, l + 64, l + 96), flips the signs, runs the unnormalised
+// Mapping: a warp takes 32 consecutive blocks (one contiguous input range).
+// Eight blocks at a time it loads them (lane l: elements l, l + 32, l + 64,
+// l + 96 of each), then block by block flips the signs, runs the unnormalised
 // WHT (two in-lane stages, five shuffle stages), reduces the squared norm and
 // writes u to shared memory, one row per block (stride 129 floats, so both
-// these row writes and the per-lane row reads below are bank-conflict free).  Then lane i searches block i:
-// per step the nearest level of each subset and its squared error, four
-// add-compare-selects (4 decision bits per step, in shared memory), then the
-// traceback, which rebuilds the pair fields in registers and stores them.
+// these row writes and the per-lane row reads below are bank-conflict free).
+// Then lane i searches block i: per step the nearest level of each subset and
+// its squared error, four add-compare-selects (4 decision bits per step, in
+// shared memory), then the traceback, which takes each step's level index
+// from its subset's decision points and rebuilds the pair fields in
+// registers.
 
 #include <cuda_fp16.h>
 
@@ -159,11 +162,13 @@ encode_v2_kernel(const __grid_constant__ EncodeParams p) {
 
   const long long item = first + lane;
   if (item >= n_items) return;
-  const long long row = item / nb;
-  const int blk = (int)(item % nb);
-  const int t = (int)(row % p.seq_new);
-  const long long bh = row / p.seq_new;
-  const int b = (int)(bh / p.kv_heads);
+  // the host keeps the item count below 2^31: 32-bit splits by multiply-high
+  const int lnb = nb == 1 ? 0 : nb == 2 ? 1 : 2;  // nb is 1, 2 or 4
+  const uint32_t row = (uint32_t)item >> lnb;
+  const int blk = (int)(item & (nb - 1));
+  const uint32_t bh = p.div_seq_new.div(row);
+  const int t = (int)(row - bh * (uint32_t)p.seq_new);
+  const int b = (int)p.div_kv_heads.div(bh);
   int pos = t;
   if (p.start_pos) pos += __ldg(p.start_pos + b);
   if (pos < 0 || pos >= p.seq_cap) {
@@ -245,8 +250,8 @@ encode_v2_kernel(const __grid_constant__ EncodeParams p) {
 template <int BITS, bool F16>
 int launch_v2_typed(const EncodeParams& p, cudaStream_t stream) {
   const long long items = (long long)p.batch * p.kv_heads * p.seq_new * (p.head_dim / kBlock);
+  if (items >= (1LL << 31)) return TQ_ERR_UNSUPPORTED;  // 32-bit index splits in the kernel
   const long long ctas = (items + kV2Threads - 1) / kV2Threads;
-  if (ctas > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
   encode_v2_kernel<BITS, F16><<<(unsigned)ctas, kV2Threads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

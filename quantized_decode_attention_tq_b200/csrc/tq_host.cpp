@@ -453,6 +453,8 @@ int tq_encode_kv_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, const tq_co
   p.norms[1] = v_norms;
   p.bits[1] = desc->v_bits;
   for (int j = 0; j < (2 << desc->v_bits); ++j) p.tcq_levels[j] = v_tcq->centroids[j];
+  p.div_seq_new = tq::FastDiv::make((uint32_t)seq_new);
+  p.div_kv_heads = tq::FastDiv::make((uint32_t)desc->kv_heads);
   p.start_pos = start_pos;
   p.status = dev_status;
   sign_mask(desc->sign_seed, p.sign_mask);
