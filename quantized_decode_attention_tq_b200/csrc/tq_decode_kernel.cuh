@@ -919,17 +919,18 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
   // ---- query preparation: qhat = H.(s o q) (D1), as this lane's fp16 MMA
   // B fragments plus the per-column score multipliers.  One warp per head
   // row: lane l holds dims 4l..4l+3 of every 128-block.  Uses res as scratch.
-  auto prep_q = [&](int b, int h0, int Gu, uint32_t (&qf)[NB][8][2], float (&qmul)[2]) {
-    constexpr int kQRows = kDup ? 4 : kMaxGroup;
-    float* qs = res;  // [kQRows] rows of scaled qhat (QScratch layout)
-    for (int j = cw; j < kQRows; j += kCWarps) {
-      float v[NB][4];
+  // The raw query row of this warp (row j = cw of the unit, warps below the
+  // row count), loaded at the segment start ahead of the tile copies so that
+  // its latency overlaps them.
+  constexpr int kQRows = kDup ? 4 : kMaxGroup;
+  auto load_q_row = [&](int b, int h0, int Gu, float (&v)[NB][4]) {
+    const int j = cw;
 #pragma unroll
-      for (int blk = 0; blk < NB; ++blk) {
+    for (int blk = 0; blk < NB; ++blk) {
+      v[blk][0] = v[blk][1] = v[blk][2] = v[blk][3] = 0.0f;
+      if (j < kQRows && j < Gu) {
         const size_t qi = vrow(b, h0 + j) * D + blk * kBlock + 4 * lane;
-        if (j >= Gu) {
-          v[blk][0] = v[blk][1] = v[blk][2] = v[blk][3] = 0.0f;
-        } else if (p.q_f16) {
+        if (p.q_f16) {
           const uint2 h = *reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(p.q) + qi);
           const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
           const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
@@ -938,11 +939,19 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
           const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.q) + qi);
           v[blk][0] = a.x; v[blk][1] = a.y; v[blk][2] = a.z; v[blk][3] = a.w;
         }
-        const uint32_t sgn = p.sign_mask[lane >> 3] >> (4 * (lane & 7));  // signs of dims 4l..4l+3
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if ((sgn >> k) & 1u) v[blk][k] = -v[blk][k];
       }
+    }
+  };
+  auto prep_q = [&](const float (&qrow)[NB][4], uint32_t (&qf)[NB][8][2], float (&qmul)[2]) {
+    float* qs = res;  // [kQRows] rows of scaled qhat (QScratch layout)
+    if (cw < kQRows) {
+      const int j = cw;
+      float v[NB][4];
+      const uint32_t sgn = p.sign_mask[lane >> 3] >> (4 * (lane & 7));  // signs of dims 4l..4l+3
+#pragma unroll
+      for (int blk = 0; blk < NB; ++blk)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[blk][k] = ((sgn >> k) & 1u) ? -qrow[blk][k] : qrow[blk][k];
       wht_rows<NB>(v, lane);
       // power-of-two scale per head so fp16 fragments neither overflow nor
       // fall into subnormals
@@ -1076,6 +1085,11 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
       if (++islot == depth) islot = 0;
     };
 
+    // this warp's query row, loaded now: its latency overlaps the append and
+    // the first copies
+    float qrow[NB][4];
+    if constexpr (HASK) load_q_row(b, h0, Gu, qrow);
+
     // ---- decode step: the CTA that holds a unit's last tile first writes the
     // sequence's new token (position len - 1) into the cache, K and V, one
     // warp per 128-block, so that its own copies read it.  Other head groups
@@ -1104,7 +1118,7 @@ decode_kernel(const __grid_constant__ DecodeParams p, int p1_ctas) {
     uint32_t qf[NB][8][2];
     float qmul[2] = {0.0f, 0.0f};
     float lse2[2] = {0.0f, 0.0f}, moff2[2] = {0.0f, 0.0f};
-    if constexpr (HASK) prep_q(b, h0, Gu, qf, qmul);
+    if constexpr (HASK) prep_q(qrow, qf, qmul);
     if constexpr (MODE == kSparseV) {
       // log-sum-exp (log2 domain) of every head of this unit, from the
       // partials that pass 1 (p1_ctas CTAs) wrote; warp hd takes head hd
