@@ -301,37 +301,65 @@ class StepBench:
         for c in range(self.n_copies):  # eager warm-up (also primes the launch caches)
             self.step(c)
         torch.cuda.synchronize()
-        self.graphs = []
-        s = torch.cuda.Stream(device=dev)
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            for c in range(self.n_copies):
-                gs = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(gs, stream=s):
-                    self.step(c)
-                self.graphs.append(gs)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
+        # Steps run as CUDA graphs of consecutive steps over the copies 0, 1,
+        # ..., so the decode launches of one graph follow one another with
+        # programmatic dependent launch (a graph launch itself waits for the
+        # one before it).  A run of n steps replays whole chunks, then a graph
+        # of the remaining steps; every graph starts at copy 0 and a chunk ends
+        # at the last copy.
+        self.chunk = self.n_copies * max(1, 64 // self.n_copies)
+        self.seq_graphs = {}
 
     def step(self, c):
         w = self.w
         self.tq.decode_step(self.caches[c], self.kcb, self.vcb, self.q, self.k_new, self.v_new, self.lens,
                             w.scale, self.out, self.ws, sparse_thr=w.sparse_thr)
 
-    def replay(self, i):
-        self.graphs[i % self.n_copies].replay()
+    def _graph(self, n):
+        """The CUDA graph of n consecutive steps (copies 0, 1, ... in turn)."""
+        g = self.seq_graphs.get(n)
+        if g is None:
+            torch = self.torch
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream(device=self.dev)
+            s.wait_stream(torch.cuda.current_stream())
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for i in range(n):
+                        self.step(i % self.n_copies)
+            torch.cuda.current_stream().wait_stream(s)
+            torch.cuda.synchronize()
+            self.seq_graphs[n] = g
+        return g
+
+    def prepare(self, n):
+        """Capture, ahead of any timed region, the graphs that run(n) replays,
+        and launch each new one once (its first launch also uploads it)."""
+        for m in ([self.chunk] if n >= self.chunk else []) + ([n % self.chunk] if n % self.chunk else []):
+            if m not in self.seq_graphs:
+                self._graph(m).replay()
+                self.torch.cuda.synchronize()
+
+    def run(self, n):
+        """n steps back to back on the current stream."""
+        full, rest = divmod(n, self.chunk)
+        for _ in range(full):
+            self._graph(self.chunk).replay()
+        if rest:
+            self._graph(rest).replay()
 
     def time_steps(self, n, warmup=3):
-        """Mean device time of one step over n graph replays (CUDA events)."""
+        """Mean device time of one step over n steps (CUDA events)."""
         torch = self.torch
-        for i in range(warmup):
-            self.replay(i)
+        self.prepare(warmup)
+        self.prepare(n)
+        self.run(warmup)
         torch.cuda.synchronize()
         stream = torch.cuda.current_stream()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(n):
-            self.replay(i)
+        self.run(n)
         e1.record(stream)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
@@ -343,7 +371,7 @@ class StepBench:
                 "frac_of_measured_hbm": gbs / peak, "kv_tokens_per_s": float(np.sum(self.w.seq_lens)) / (ms / 1e3)}
 
     def release(self):
-        self.graphs = []
+        self.seq_graphs = {}
         self.caches = []
         self.cache0 = None
         self.torch.cuda.synchronize()
@@ -500,8 +528,9 @@ def run_tq(args):
     peak, peak_kind = measured_peaks()
     sb = StepBench(args.workload, dev, tqd.workload_seed(rank))
     w, n_copies = sb.w, sb.n_copies
-    for i in range(args.warmup):
-        sb.replay(i)
+    sb.prepare(args.warmup)
+    sb.prepare(args.steps)
+    sb.run(args.warmup)
     torch.cuda.synchronize()
 
     # ---- timed region: exactly `steps` steps back to back (one CUDA event
@@ -514,8 +543,7 @@ def run_tq(args):
     sampler = ClockSampler(local)
     time.sleep(0.3)
     ev0.record(stream)
-    for i in range(args.steps):
-        sb.replay(i)
+    sb.run(args.steps)
     ev1.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -533,14 +561,15 @@ def run_tq(args):
     sustained = None
     if args.sustain_s > 0:
         n_long = max(args.steps, int(math.ceil(args.sustain_s / max(ms / 1e3, 1e-6))))
+        n_long = (n_long + sb.chunk - 1) // sb.chunk * sb.chunk  # whole chunks
+        sb.prepare(n_long)
         barrier()
         torch.cuda.synchronize()
         sampler2 = ClockSampler(local)
         time.sleep(0.3)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record(stream)
-        for i in range(n_long):
-            sb.replay(i)
+        sb.run(n_long)
         s1.record(stream)
         torch.cuda.synchronize()
         clocks2 = sampler2.stop()
