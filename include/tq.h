@@ -24,6 +24,16 @@
  *   - Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *     default stream).  Device work is asynchronous on that stream; only
  *     tq_make_codebook and tq_sign_vector are synchronous (host only).
+ *   - Launch overlap: the decode entry points without sparse-V launch with
+ *     programmatic stream serialisation, so a decode launch may start while
+ *     the kernel before it in the stream is still running if that kernel
+ *     signals its dependents early (griddepcontrol.launch_dependents /
+ *     cudaTriggerProgrammaticLaunchCompletion; of this library's kernels only
+ *     the decode kernel does).  The launch reads `seq_lens` before it waits
+ *     for that kernel and everything else (query, cache, new rows, workspace,
+ *     output) after: a preceding kernel that signals early must not write
+ *     `seq_lens` after its signal.  After any other kernel, a copy or an
+ *     event wait the launch starts as an ordinary one.
  *   - Errors: every call returns a tq_status code and never throws.  Host-side
  *     validation runs first; when it fails nothing is launched.  Range errors
  *     that only the device can see (a position or a length outside the cache,
