@@ -181,12 +181,13 @@ __device__ __forceinline__ uint2 ld_table2(uint32_t a) {
 //    put in bits 8..15 of this lane's base word by one byte permute.
 
 // Address of the 3-bit pair whose field starts at bit `pos` of the word array
-// w: the field shifted to bit 7 (one funnel shift when it continues in the
-// next word), then the mask and the lane base in one three-input logic op.
+// w: the field shifted to bit 7 (one funnel shift by pos - 7 when it continues
+// in the next word: such a field starts at bit 27 or later), then the mask and
+// the lane base in one three-input logic op.
 __device__ __forceinline__ uint32_t addr3(const uint32_t* w, int pos, uint32_t lb) {
   const int wi = pos >> 5, sh = pos & 31;
   uint32_t x;
-  if (sh + 6 > 32) x = __funnelshift_r(w[wi], w[wi + 1], sh) << 7;
+  if (sh + 6 > 32) x = __funnelshift_r(w[wi], w[wi + 1], sh - 7);
   else x = sh >= 7 ? w[wi] >> (sh - 7) : w[wi] << (7 - sh);
   return (x & (63u << 7)) | lb;
 }
