@@ -259,7 +259,7 @@ def run_reference(args):
 class StepBench:
     """One workload on one GPU: its packed cache (built by the library's
     encoder) in enough copies that every step reads cold memory, the step's
-    device inputs, and one CUDA graph per copy holding the step's launch(es).
+    device inputs, and CUDA graphs of consecutive steps over the copies.
 
     A step is one decode step of every sequence: the newest K/V row is encoded
     into the cache at seq_len - 1 inside the decode launch, then attention runs
