@@ -423,6 +423,32 @@ int tq_decode_attention_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, cons
                            const int32_t* seq_lens, float scale, float sparse_thr, float* out,
                            void* workspace, size_t workspace_bytes, uint32_t* dev_status, void* stream);
 
+/*
+ * tq_decode_attention_multi_v3, tq_decode_attention_multi_v2 -- multi-token
+ * queries (tq_decode_attention_multi) over a v3 or a v2 V cache: query token
+ * j of sequence b sees positions [0, seq_lens[b] - n_q + j], and its output
+ * is that of tq_decode_attention_v3 / tq_decode_attention_v2 over that range.
+ * q and out are [batch, n_q, q_heads, head_dim]; the workspace is
+ * tq_decode_workspace_size(desc, q_heads * n_q, sparse_thr) bytes.  Every
+ * other argument, limit and error is that of the single-token entry point of
+ * the same format and of tq_decode_attention_multi (n_q = 1 gives exactly
+ * the single-token results).
+ */
+int tq_decode_attention_multi_v3(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                                 const tq_codebook* v_cb, int q_heads, int n_q, const void* q,
+                                 int q_dtype, const uint8_t* k_codes, const uint16_t* k_norms,
+                                 const uint8_t* v_codes, const uint16_t* v_norms,
+                                 const tq_v_outliers* vo, const int32_t* seq_lens, float scale,
+                                 float sparse_thr, float* out, void* workspace,
+                                 size_t workspace_bytes, uint32_t* dev_status, void* stream);
+int tq_decode_attention_multi_v2(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                                 const tq_codebook* v_tcq, int q_heads, int n_q, const void* q,
+                                 int q_dtype, const uint8_t* k_codes, const uint16_t* k_norms,
+                                 const uint8_t* v_codes, const uint16_t* v_norms,
+                                 const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                                 void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                                 void* stream);
+
 /* Static description of a status code. */
 const char* tq_status_string(int status);
 

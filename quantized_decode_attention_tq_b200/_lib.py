@@ -70,6 +70,14 @@ SIGNATURES = {
     "tq_decode_attention_v3": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_void_p, c_int,
                                        c_void_p, c_void_p, c_void_p, c_void_p, _P(VOutliers), c_void_p,
                                        c_float, c_float, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "tq_decode_attention_multi_v3": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_int,
+                                             c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             _P(VOutliers), c_void_p, c_float, c_float, c_void_p, c_void_p,
+                                             c_size_t, c_void_p, c_void_p]),
+    "tq_decode_attention_multi_v2": (c_int, [_P(KVDesc), _P(Codebook), _P(Codebook), c_int, c_int,
+                                             c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                             c_void_p, c_float, c_float, c_void_p, c_void_p, c_size_t,
+                                             c_void_p, c_void_p]),
     "tq_status_string": (ctypes.c_char_p, [c_int]),
 }
 

@@ -283,6 +283,24 @@ def decode_attention_v3(cache: Cache, k_cb: Codebook, v_cb: Codebook, vo: VOutli
     return out
 
 
+def decode_attention_multi_v3(cache: Cache, k_cb: Codebook, v_cb: Codebook, vo: VOutliers, q, seq_lens,
+                              scale: float, out, workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """decode_attention_multi over a v3 V cache (tq_decode_attention_multi_v3).
+    q, out: [B, n_q, Hq, D]; workspace: alloc_workspace(desc, Hq * n_q, sparse_thr)."""
+    vs = vo.c_struct()
+    n_q, q_heads = q.shape[1], q.shape[2]
+    st = lib().tq_decode_attention_multi_v3(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_cb), q_heads, n_q,
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"), ctypes.byref(vs),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention_multi_v3", st)
+    return out
+
+
 # ---- V v2: trellis-coded quantisation --------------------------------------
 
 def make_tcq_codebook(v_bits: int) -> Codebook:
@@ -322,4 +340,21 @@ def decode_attention_v2(cache: Cache, k_cb: Codebook, v_tcq: Codebook, q, seq_le
         _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(status, "status"), _stream(stream))
     check("tq_decode_attention_v2", st)
+    return out
+
+
+def decode_attention_multi_v2(cache: Cache, k_cb: Codebook, v_tcq: Codebook, q, seq_lens, scale: float, out,
+                              workspace, sparse_thr: float = 0.0, status=None, stream=None):
+    """decode_attention_multi over a v2 V cache (tq_decode_attention_multi_v2).
+    q, out: [B, n_q, Hq, D]; workspace: alloc_workspace(desc, Hq * n_q, sparse_thr)."""
+    n_q, q_heads = q.shape[1], q.shape[2]
+    st = lib().tq_decode_attention_multi_v2(
+        ctypes.byref(cache.desc), ctypes.byref(k_cb), ctypes.byref(v_tcq), q_heads, n_q,
+        _ptr(q, "q"), _dtype_code(q),
+        _ptr(cache.k_codes, "k_codes"), _ptr(cache.k_norms, "k_norms"),
+        _ptr(cache.v_codes, "v_codes"), _ptr(cache.v_norms, "v_norms"),
+        _ptr(seq_lens, "seq_lens"), float(scale), float(sparse_thr), _ptr(out, "out"),
+        _ptr(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(status, "status"), _stream(stream))
+    check("tq_decode_attention_multi_v2", st)
     return out

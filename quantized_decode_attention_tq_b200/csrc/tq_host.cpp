@@ -477,6 +477,30 @@ int tq_decode_attention_v2(const tq_kv_desc* desc, const tq_codebook* k_cb, cons
                        nullptr, nullptr, 2);
 }
 
+int tq_decode_attention_multi_v3(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                                 const tq_codebook* v_cb, int q_heads, int n_q, const void* q,
+                                 int q_dtype, const uint8_t* k_codes, const uint16_t* k_norms,
+                                 const uint8_t* v_codes, const uint16_t* v_norms,
+                                 const tq_v_outliers* vo, const int32_t* seq_lens, float scale,
+                                 float sparse_thr, float* out, void* workspace,
+                                 size_t workspace_bytes, uint32_t* dev_status, void* stream) {
+  return decode_common(desc, k_cb, v_cb, q_heads, n_q, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       nullptr, vo);
+}
+
+int tq_decode_attention_multi_v2(const tq_kv_desc* desc, const tq_codebook* k_cb,
+                                 const tq_codebook* v_tcq, int q_heads, int n_q, const void* q,
+                                 int q_dtype, const uint8_t* k_codes, const uint16_t* k_norms,
+                                 const uint8_t* v_codes, const uint16_t* v_norms,
+                                 const int32_t* seq_lens, float scale, float sparse_thr, float* out,
+                                 void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                                 void* stream) {
+  return decode_common(desc, k_cb, v_tcq, q_heads, n_q, q, q_dtype, k_codes, k_norms, v_codes, v_norms,
+                       seq_lens, scale, sparse_thr, out, workspace, workspace_bytes, dev_status, stream,
+                       nullptr, nullptr, 2);
+}
+
 int tq_pick_outlier_channels(const tq_kv_desc* desc, const void* v, int v_dtype, int rows, int k,
                              int32_t* channels, void* stream) {
   int st = check_desc(desc);

@@ -94,3 +94,63 @@ def test_decode_multi_sixteen_tokens():
     # the largest n_q the ABI accepts: 64 (token, head) columns per kv-head
     w = inputs.make("gqa", batch=2, seq=256)
     _check(w, tq._lib.TQ_MAX_QUERY_TOKENS, [256, 90], seed=16)
+
+
+# ---- multi-token queries over v3 and v2 V caches ---------------------------
+
+def _multi_fmt(fn, cache, kcb, vcb, q, lens, scale, *extra):
+    torch = torch_mod()
+    B, n_q, hq, D = q.shape
+    out = torch.full((B, n_q, hq, D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = tq.alloc_workspace(cache.desc, hq * n_q, 0.0)
+    fn(cache, kcb, vcb, *extra, to_dev(q), to_dev(np.asarray(lens, dtype=np.int32)), scale, out, ws)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("n_q,lens", [(2, [400, 251]), (3, [400, 3])])
+def test_decode_multi_v3(n_q, lens):
+    """Token j over a v3 cache equals the single-token v3 oracle over the first
+    len - n_q + j + 1 positions (outlier channels and the rest each within the
+    decode tolerance); n_q = 1 is tq_decode_attention_v3 bit for bit."""
+    from .test_v3_gpu import _check_v3_decode, _decode_v3, _encode_v3
+    w = inputs.make("gqa", batch=2, seq=400, dist="outlier_v")
+    rng = np.random.default_rng(40 + n_q)
+    q = rng.standard_normal((2, n_q, w.q_heads, w.head_dim)).astype(np.float16)
+    cache, kcb, vcb, vo = _encode_v3(w, 8)
+    o = _multi_fmt(tq.decode_attention_multi_v3, cache, kcb, vcb, q, lens, w.scale, vo)
+    kc, kn, vc, vn = host(cache)
+    vals = vo.values.cpu().numpy().view(np.float16)[..., : vo.k]
+    ch = vo.channels.cpu().numpy()
+    kcent, vcent = O.codebook_f32(w.k_bits)[0], O.codebook_f32(w.v_bits)[0]
+    for j in range(n_q):
+        lj = np.maximum(np.asarray(lens) - n_q + j + 1, 0)
+        ref = O.decode_v3_rotated(q[:, j].astype(np.float64), kc, kn, vc, vn, vals, ch, lj, w.scale, w.k_bits,
+                                  w.v_bits, kcent, vcent, O.sign_vector(w.sign_seed), 0.0)
+        _check_v3_decode(o[:, j], ref, ch, w.q_heads // w.kv_heads)
+    one = _multi_fmt(tq.decode_attention_multi_v3, cache, kcb, vcb, q[:, :1], lens, w.scale, vo)
+    single = _decode_v3(cache, kcb, vcb, vo, q[:, 0], lens, w.scale)
+    assert np.array_equal(one[:, 0], single)
+
+
+@pytest.mark.parametrize("n_q,lens,vb", [(2, [400, 251], 3), (3, [400, 3], 2)])
+def test_decode_multi_v2(n_q, lens, vb):
+    """Token j over a v2 cache equals the single-token v2 oracle over the first
+    len - n_q + j + 1 positions; n_q = 1 is tq_decode_attention_v2 bit for bit."""
+    from .test_v2_gpu import _decode_v2, _encode_v2
+    w = inputs.make("gqa", batch=2, seq=400)
+    w.v_bits = vb
+    rng = np.random.default_rng(50 + n_q)
+    q = rng.standard_normal((2, n_q, w.q_heads, w.head_dim)).astype(np.float16)
+    cache, kcb, vtq = _encode_v2(w)
+    o = _multi_fmt(tq.decode_attention_multi_v2, cache, kcb, vtq, q, lens, w.scale)
+    kc, kn, vc, vn = host(cache)
+    for j in range(n_q):
+        lj = np.maximum(np.asarray(lens) - n_q + j + 1, 0)
+        ref = O.decode_v2_rotated(q[:, j].astype(np.float64), kc, kn, vc, vn, lj, w.scale, w.k_bits, w.v_bits,
+                                  O.codebook_f32(w.k_bits)[0], O.tcq_levels_f32(w.v_bits),
+                                  O.sign_vector(w.sign_seed), 0.0)
+        check_decode(o[:, j], ref)
+    one = _multi_fmt(tq.decode_attention_multi_v2, cache, kcb, vtq, q[:, :1], lens, w.scale)
+    single = _decode_v2(cache, kcb, vtq, q[:, 0], lens, w.scale)
+    assert np.array_equal(one[:, 0], single)

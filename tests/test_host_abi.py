@@ -24,7 +24,7 @@ def _header_functions():
 
 def test_library_exports_every_declared_symbol():
     names = _header_functions()
-    assert len(names) == 15
+    assert len(names) == 17
     lib = tq.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -346,3 +346,33 @@ def test_v2_entry_points_reject_bad_arguments_without_launch():
     assert dec(d2, tq.make_codebook(2)) == _lib.TQ_ERR_INVALID_ARG
     assert dec(tq.kv_desc(2, 2, 128, 64, 3, 4), tq.make_codebook(4)) == _lib.TQ_ERR_UNSUPPORTED
     assert dec(d2, tq.make_tcq_codebook(2), wsb=16) == _lib.TQ_ERR_WORKSPACE
+
+
+def test_multi_token_v3_v2_reject_bad_arguments_without_launch():
+    lib = tq.lib()
+    d = tq.kv_desc(2, 2, 128, 64, 3, 2)
+    cb3, cb2, vtq = tq.make_codebook(3), tq.make_codebook(2), tq.make_tcq_codebook(2)
+
+    def v3(n_q, vo, wsb=None):
+        need = tq.decode_workspace_size(d, 8 * max(n_q, 1)) if wsb is None else wsb
+        return lib.tq_decode_attention_multi_v3(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(cb2), 8, n_q,
+                                                _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                                _fake(GOOD), ctypes.byref(vo), _fake(GOOD), 0.1, 0.0, _fake(GOOD),
+                                                _fake(GOOD), need, None, None)
+
+    def v2(n_q, vcb, wsb=None):
+        need = tq.decode_workspace_size(d, 8 * max(n_q, 1)) if wsb is None else wsb
+        return lib.tq_decode_attention_multi_v2(ctypes.byref(d), ctypes.byref(cb3), ctypes.byref(vcb), 8, n_q,
+                                                _fake(GOOD), 1, _fake(GOOD), _fake(GOOD), _fake(GOOD),
+                                                _fake(GOOD), _fake(GOOD), 0.1, 0.0, _fake(GOOD), _fake(GOOD),
+                                                need, None, None)
+
+    for n_q in (0, _lib.TQ_MAX_QUERY_TOKENS + 1):
+        assert v3(n_q, _vo()) == _lib.TQ_ERR_INVALID_ARG
+        assert v2(n_q, vtq) == _lib.TQ_ERR_INVALID_ARG
+    assert v3(4, _vo(k=17)) == _lib.TQ_ERR_INVALID_ARG                       # the v3 checks
+    assert v2(4, cb2) == _lib.TQ_ERR_INVALID_ARG                             # V needs the doubled codebook
+    # the workspace must be sized for q_heads * n_q
+    assert v3(4, _vo(), wsb=tq.decode_workspace_size(d, 8)) == _lib.TQ_ERR_WORKSPACE
+    assert v2(4, vtq, wsb=tq.decode_workspace_size(d, 8)) == _lib.TQ_ERR_WORKSPACE
+
