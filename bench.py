@@ -256,6 +256,12 @@ def run_reference(args):
     return 0
 
 
+def graph_plan(n, chunk):
+    """Lengths of the step graphs that run n steps: whole chunks, then the rest."""
+    full, rest = divmod(n, chunk)
+    return [chunk] * full + ([rest] if rest else [])
+
+
 class StepBench:
     """One workload on one GPU: its packed cache (built by the library's
     encoder) in enough copies that every step reads cold memory, the step's
@@ -336,18 +342,15 @@ class StepBench:
     def prepare(self, n):
         """Capture, ahead of any timed region, the graphs that run(n) replays,
         and launch each new one once (its first launch also uploads it)."""
-        for m in ([self.chunk] if n >= self.chunk else []) + ([n % self.chunk] if n % self.chunk else []):
+        for m in sorted(set(graph_plan(n, self.chunk))):
             if m not in self.seq_graphs:
                 self._graph(m).replay()
                 self.torch.cuda.synchronize()
 
     def run(self, n):
         """n steps back to back on the current stream."""
-        full, rest = divmod(n, self.chunk)
-        for _ in range(full):
-            self._graph(self.chunk).replay()
-        if rest:
-            self._graph(rest).replay()
+        for m in graph_plan(n, self.chunk):
+            self._graph(m).replay()
 
     def time_steps(self, n, warmup=3):
         """Mean device time of one step over n steps (CUDA events)."""

@@ -35,3 +35,19 @@ def test_gpus_must_match_the_launched_world():
                         "--warmup", "0"], capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
     assert r.returncode != 0
     assert "--gpus 2 but the launcher started 1 rank" in r.stderr
+
+
+def test_step_graphs_run_exactly_the_requested_steps():
+    """The timed region replays graphs of consecutive steps: whole chunks, then
+    one graph of the rest, so exactly n steps run and every graph starts at
+    cache copy 0 after a graph that ended at the last copy."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for copies in (2, 3, 5):
+        chunk = copies * max(1, 64 // copies)
+        assert chunk % copies == 0
+        for n in (0, 1, 3, 20, chunk - 1, chunk, chunk + 1, 3 * chunk + 7, 11088):
+            plan = bench.graph_plan(n, chunk)
+            assert sum(plan) == n
+            assert all(0 < m <= chunk for m in plan)
+            assert all(m == chunk for m in plan[:-1])   # only the last graph is short
